@@ -1,0 +1,188 @@
+"""Exact IO-aware attention for B200: thin Python binding of the C-ABI library
+``libattn.so`` (declared in ``include/attn.h``).
+
+This module only marshals arguments: it checks shapes/dtypes, allocates the
+output tensors with PyTorch (device memory and streams are PyTorch's), and
+calls the C entry points of the same names.  Every step of the attention path
+runs in the library's CUDA kernels; there is no fallback.  If the library is
+missing, importing this module raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+from pathlib import Path
+
+import torch
+
+_PKG = Path(__file__).resolve().parent
+LIB_PATH = _PKG / "libattn.so"
+
+ATTN_BF16 = 0
+ATTN_F32 = 1
+ATTN_OK = 0
+ATTN_ERR_INVALID = -1
+ATTN_ERR_UNSUPPORTED = -2
+ATTN_ERR_WORKSPACE = -3
+ATTN_ERR_CUDA = -4
+ATTN_ERR_TIMEOUT = -5
+
+# symbol -> (restype, argtypes)
+_VP, _FP, _IP = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p
+_I, _LL, _F, _SZ = ctypes.c_int, ctypes.c_longlong, ctypes.c_float, ctypes.c_size_t
+EXPORTS = {
+    "attn_fwd": (_I, [_VP, _VP, _VP, _FP, _LL, _VP, _FP, _I, _I, _I, _I, _I, _I, _F, _I, _I, _VP]),
+    "attn_bwd_workspace_size": (_SZ, [_I, _I, _I, _I]),
+    "attn_bwd": (_I, [_VP, _VP, _VP, _FP, _LL, _VP, _FP, _VP, _VP, _VP, _VP, _VP, _SZ, _I, _I, _I, _I, _I,
+                      _I, _F, _I, _I, _VP]),
+    "attn_fwd_varlen": (_I, [_VP, _VP, _VP, _VP, _FP, _IP, _IP, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I, _I,
+                             _VP]),
+    "attn_naive_scratch_size": (_SZ, [_I, _I]),
+    "attn_fwd_naive": (_I, [_VP, _VP, _VP, _VP, _FP, _VP, _SZ, _I, _I, _I, _I, _I, _I, _F, _I, _VP]),
+    "attn_strerror": (ctypes.c_char_p, [_I]),
+    "attn_device_status": (_I, [_VP]),
+    "attn_launch_count": (_LL, [_I]),
+}
+
+
+class AttnError(RuntimeError):
+    pass
+
+
+def _load() -> ctypes.CDLL:
+    if not LIB_PATH.exists():
+        raise ImportError(f"{LIB_PATH} is missing: build it with `python -m exact_io_aware_57_b200.build`")
+    lib = ctypes.CDLL(str(LIB_PATH))
+    for name, (res, args) in EXPORTS.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    return lib
+
+
+_lib = _load()
+
+
+def lib() -> ctypes.CDLL:
+    return _lib
+
+
+def _check(rc: int) -> None:
+    if rc != ATTN_OK:
+        raise AttnError(f"libattn error {rc}: {_lib.attn_strerror(rc).decode()}")
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return ATTN_BF16
+    if t.dtype == torch.float32:
+        return ATTN_F32
+    raise AttnError(f"unsupported dtype {t.dtype} (bf16 or fp32)")
+
+
+def _dev(t: torch.Tensor, name: str) -> int:
+    if not t.is_cuda:
+        raise AttnError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise AttnError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def _stream(stream) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return s.cuda_stream
+
+
+def _bias_args(bias, B, Hq, Nq, Nk):
+    if bias is None:
+        return None, 0
+    if bias.dtype != torch.float32:
+        raise AttnError("bias must be fp32")
+    per = Hq * Nq * Nk
+    if bias.numel() == per:
+        return _dev(bias, "bias"), 0
+    if bias.numel() == B * per:
+        return _dev(bias, "bias"), per
+    raise AttnError("bias must be [Hq,Nq,Nk] or [B,Hq,Nq,Nk]")
+
+
+def attn_fwd(q, k, v, bias=None, causal=False, scale=None, out=None, lse=None, stream=None):
+    """O, LSE = attention(q [B,Nq,Hq,d], k/v [B,Nk,Hkv,d]); o like q, lse fp32 [B,Hq,Nq]."""
+    B, Nq, Hq, d = q.shape
+    Nk, Hkv = k.shape[1], k.shape[2]
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    o = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, Hq, Nq), device=q.device, dtype=torch.float32) if lse is None else lse
+    bp, bs = _bias_args(bias, B, Hq, Nq, Nk)
+    _check(_lib.attn_fwd(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), bp, bs, _dev(o, "o"), _dev(lse, "lse"),
+                         B, Hq, Hkv, Nq, Nk, d, scale, int(bool(causal)), _dtype_code(q), _stream(stream)))
+    return o, lse
+
+
+def attn_bwd_workspace_size(batch, h_q, n_q, d) -> int:
+    return int(_lib.attn_bwd_workspace_size(batch, h_q, n_q, d))
+
+
+def attn_bwd(q, k, v, o, lse, dout, bias=None, causal=False, scale=None, workspace=None, dq=None, dk=None,
+             dv=None, stream=None):
+    """dq, dk, dv of attn_fwd for upstream gradient dout (layouts as q, k, v)."""
+    B, Nq, Hq, d = q.shape
+    Nk, Hkv = k.shape[1], k.shape[2]
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    need = attn_bwd_workspace_size(B, Hq, Nq, d)
+    if workspace is None:
+        workspace = torch.empty(need, device=q.device, dtype=torch.uint8)
+    bp, bs = _bias_args(bias, B, Hq, Nq, Nk)
+    _check(_lib.attn_bwd(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), bp, bs, _dev(o, "o"), _dev(lse, "lse"),
+                         _dev(dout, "dout"), _dev(dq, "dq"), _dev(dk, "dk"), _dev(dv, "dv"),
+                         _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(),
+                         B, Hq, Hkv, Nq, Nk, d, scale, int(bool(causal)), _dtype_code(q), _stream(stream)))
+    return dq, dk, dv
+
+
+def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, causal=False, scale=None,
+                    out=None, lse=None, stream=None):
+    """Packed forward: q [Tq,Hq,d], k/v [Tk,Hkv,d], cu_seqlens int32 device; lse [Hq,Tq]."""
+    Tq, Hq, d = q.shape
+    Tk, Hkv = k.shape[0], k.shape[1]
+    if cu_seqlens_q.dtype != torch.int32 or cu_seqlens_k.dtype != torch.int32:
+        raise AttnError("cu_seqlens must be int32")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    o = torch.empty_like(q) if out is None else out
+    lse = torch.empty((Hq, Tq), device=q.device, dtype=torch.float32) if lse is None else lse
+    _check(_lib.attn_fwd_varlen(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(o, "o"), _dev(lse, "lse"),
+                                _dev(cu_seqlens_q, "cu_seqlens_q"), _dev(cu_seqlens_k, "cu_seqlens_k"),
+                                cu_seqlens_q.numel() - 1, int(max_seqlen_q), int(max_seqlen_k), Tq, Tk, Hq, Hkv,
+                                d, scale, int(bool(causal)), _dtype_code(q), _stream(stream)))
+    return o, lse
+
+
+def attn_naive_scratch_size(n_q, n_k) -> int:
+    return int(_lib.attn_naive_scratch_size(n_q, n_k))
+
+
+def attn_fwd_naive(q, k, v, causal=False, scale=None, scratch=None, stream=None):
+    """Materialising three-step forward (measurement comparator only)."""
+    B, Nq, Hq, d = q.shape
+    Nk, Hkv = k.shape[1], k.shape[2]
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    o = torch.empty_like(q)
+    lse = torch.empty((B, Hq, Nq), device=q.device, dtype=torch.float32)
+    if scratch is None:
+        scratch = torch.empty(attn_naive_scratch_size(Nq, Nk), device=q.device, dtype=torch.uint8)
+    _check(_lib.attn_fwd_naive(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(o, "o"), _dev(lse, "lse"),
+                               _dev(scratch, "scratch"), scratch.numel(), B, Hq, Hkv, Nq, Nk, d, scale,
+                               int(bool(causal)), _stream(stream)))
+    return o, lse
+
+
+def attn_device_status(stream=None) -> int:
+    """Synchronise and return/clear the device status word (0 or ATTN_ERR_TIMEOUT)."""
+    return int(_lib.attn_device_status(_stream(stream)))
+
+
+def attn_launch_count(reset: bool = False) -> int:
+    return int(_lib.attn_launch_count(int(bool(reset))))

@@ -1,0 +1,401 @@
+// Forward attention on sm_100a tensor cores.
+//
+// One CTA owns a tile of 128 query rows of one (batch or sequence, head) and
+// streams 128-key tiles of K and V past it ("Attention IO tiling" lesson card,
+// The mechanism: partition into tiles that fit the local-memory budget, form
+// one score block, update running softmax statistics, accumulate weighted
+// values while rescaling, discard the score block).
+//
+//   warp 0      TMA producer: Q once, then K_j / V_j into a 2-stage smem ring
+//   warp 1      TMEM owner + single-thread tcgen05.mma issuer
+//   warps 2..5  softmax warpgroup: thread t owns query row t (TMEM lane t)
+//
+// TMEM (512 columns x 128 lanes x 32 bit):
+//   [  0,128) S buffer 0   [128,256) S buffer 1     (fp32 scores, S = Q K_j^T)
+//   [256,256+D) O accumulator (fp32)
+//   [384,448) P buffer 0   [448,512) P buffer 1     (bf16 pairs, A operand of P V_j)
+//
+// Per key tile j the softmax thread of row i forms t = s * scale * log2(e)
+// (+ bias * log2(e)), the new running max m' = max(m, max_j t), p = 2^(t - m'),
+// l' = 2^(m - m') l + sum p ("Softmax does not need the matrix", "Carry the
+// Normalizer", in base 2), writes P to TMEM and -- once the previous P V has
+// landed -- rescales the O accumulator by 2^(m - m') when the max moved.  The
+// MMA warp then accumulates O += P V_j.  O / l and LSE = (m + log2 l) ln 2 are
+// written once at the end ("normalize once at the end", the same page's lab).
+// Causal: KV tiles that lie wholly above the diagonal are never loaded.
+#include <algorithm>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace attn {
+
+namespace {
+
+constexpr int BM = 128;          // query rows per CTA
+constexpr int BN = 128;          // keys per KV tile
+constexpr int NST = 2;           // K/V smem stages
+constexpr int kThreads = 192;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColS = 0, kColO = 256, kColP = 384;
+
+template <int D>
+struct FwdSmem {
+  static constexpr int kTileBytes = BM * D * 2;  // 128 rows x D bf16
+  alignas(1024) uint8_t q[kTileBytes];
+  alignas(1024) uint8_t k[NST][kTileBytes];
+  alignas(1024) uint8_t v[NST][kTileBytes];
+  uint64_t q_full;
+  uint64_t k_full[NST], k_empty[NST], v_full[NST], v_empty[NST];
+  uint64_t s_full[2], s_free[2], p_full[2];
+  uint64_t pv_done, drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+struct FwdParams {
+  __nv_bfloat16* o;
+  float* lse;
+  const float* bias;
+  long long bias_bstride;
+  const int* cu_q;
+  const int* cu_k;
+  int Hq, Hkv, Nq, Nk;
+  long long o_bstride, lse_bstride, lse_hstride;
+  float scale_log2;
+  int causal;
+  int* status;
+  long long wait_limit;
+};
+
+// Keep the compiler from using TMEM-loaded registers before tcgen05.wait::ld.
+template <int N>
+ATTN_DEVINL void reg_fence(uint32_t (&r)[N]) {
+#pragma unroll
+  for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
+}
+
+template <int D, bool HAS_BIAS>
+__global__ void __launch_bounds__(kThreads, 1)
+    fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                     const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
+  using Smem = FwdSmem<D>;
+  constexpr int KB = D / 64;  // 64-column (128-byte) blocks per row
+  extern __shared__ uint8_t smem_raw[];
+  Smem& s = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  // ---- work tile: heavy (late) query tiles first under causal masking
+  const int m_tile = p.causal ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x;
+  const int h = blockIdx.y, z = blockIdx.z;
+  int q_off = 0, len_q = p.Nq, k_off = 0, len_k = p.Nk, bidx = z;
+  if (p.cu_q) {
+    q_off = p.cu_q[z];
+    len_q = p.cu_q[z + 1] - q_off;
+    k_off = p.cu_k[z];
+    len_k = p.cu_k[z + 1] - k_off;
+    bidx = 0;
+  }
+  const int m0 = m_tile * BM;
+  if (m0 >= len_q) return;  // uniform: before any barrier or TMEM use
+  const int hk = h / (p.Hq / p.Hkv);
+  const int diag = len_k - len_q;  // key j visible from row i iff j <= i + diag
+  int kv_end = len_k;
+  if (p.causal) kv_end = min(len_k, m0 + BM + diag);
+  const int n_kv = kv_end > 0 ? (kv_end + BN - 1) / BN : 0;
+
+  // ---- setup
+  if (threadIdx.x == 0) {
+    s.abort_flag = 0;
+    mbar_init(&s.q_full, 1);
+    for (int i = 0; i < NST; ++i) {
+      mbar_init(&s.k_full[i], 1);
+      mbar_init(&s.k_empty[i], 1);
+      mbar_init(&s.v_full[i], 1);
+      mbar_init(&s.v_empty[i], 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s.s_full[i], 1);
+      mbar_init(&s.s_free[i], 4);
+      mbar_init(&s.p_full[i], 4);
+    }
+    mbar_init(&s.pv_done, 1);
+    mbar_init(&s.drain, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(&s.tmem_base, kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s.tmem_base;
+  const Abort ab{&s.abort_flag, p.status, p.wait_limit};
+
+  if (warp == 0) {
+    // ===================================================== TMA producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      mbar_expect_tx(&s.q_full, Smem::kTileBytes);
+#pragma unroll
+      for (int kb = 0; kb < KB; ++kb)
+        tma_load_4d(s.q + kb * BM * 128, &tm_q, &s.q_full, kb * 64, h, q_off + m0, bidx);
+      int issued_k = 0, issued_v = 0;
+      for (int j = 0; j < n_kv; ++j) {
+        const int st = j % NST;
+        const uint32_t ph = (j / NST) & 1;
+        if (!mbar_wait(&s.k_empty[st], ph ^ 1, ab)) break;
+        mbar_expect_tx(&s.k_full[st], Smem::kTileBytes);
+#pragma unroll
+        for (int kb = 0; kb < KB; ++kb)
+          tma_load_4d(s.k[st] + kb * BN * 128, &tm_k, &s.k_full[st], kb * 64, hk, k_off + j * BN, bidx);
+        ++issued_k;
+        if (!mbar_wait(&s.v_empty[st], ph ^ 1, ab)) break;
+        mbar_expect_tx(&s.v_full[st], Smem::kTileBytes);
+#pragma unroll
+        for (int kb = 0; kb < KB; ++kb)
+          tma_load_4d(s.v[st] + kb * BN * 128, &tm_v, &s.v_full[st], kb * 64, hk, k_off + j * BN, bidx);
+        ++issued_v;
+      }
+      if (s.abort_flag) {
+        // leave no copy in flight into shared memory that is about to be released
+        mbar_wait_drain(&s.q_full, 0, p.wait_limit);
+        for (int j = max(0, issued_k - NST); j < issued_k; ++j)
+          mbar_wait_drain(&s.k_full[j % NST], (j / NST) & 1, p.wait_limit);
+        for (int j = max(0, issued_v - NST); j < issued_v; ++j)
+          mbar_wait_drain(&s.v_full[j % NST], (j / NST) & 1, p.wait_limit);
+      }
+    }
+  } else if (warp == 1) {
+    // ===================================================== MMA issuer
+    if (lane == 0 && n_kv > 0) {
+      constexpr uint32_t idesc_s = idesc_bf16(BM, BN, 0, 0);   // Q: K-major, K_j: K-major
+      constexpr uint32_t idesc_pv = idesc_bf16(BM, D, 0, 1);   // P: TMEM, V_j: MN-major
+      const uint32_t q_addr = smem_u32(s.q);
+      auto issue_s = [&](int j) -> bool {
+        const int buf = j & 1, st = j % NST;
+        if (j >= 2 && !mbar_wait(&s.s_free[buf], ((j >> 1) - 1) & 1, ab)) return false;
+        if (!mbar_wait(&s.k_full[st], (j / NST) & 1, ab)) return false;
+        tc_fence_after();
+        const uint32_t k_addr = smem_u32(s.k[st]);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
+          mma_ss(tmem + kColS + buf * BN, sdesc_sw128(q_addr + off, 16, 1024), sdesc_sw128(k_addr + off, 16, 1024),
+                 idesc_s, kk > 0);
+        }
+        mma_commit(&s.s_full[buf]);
+        mma_commit(&s.k_empty[st]);
+        return true;
+      };
+      bool ok = mbar_wait(&s.q_full, 0, ab);
+      if (ok) ok = issue_s(0);
+      if (ok && n_kv > 1) ok = issue_s(1);
+      for (int j = 0; ok && j < n_kv; ++j) {
+        const int buf = j & 1, st = j % NST;
+        if (!mbar_wait(&s.p_full[buf], (j >> 1) & 1, ab)) break;
+        if (!mbar_wait(&s.v_full[st], (j / NST) & 1, ab)) break;
+        tc_fence_after();
+        const uint32_t v_addr = smem_u32(s.v[st]);
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk)
+          mma_ts(tmem + kColO, tmem + kColP + buf * 64 + kk * 8, sdesc_sw128(v_addr + kk * 2048, BN * 128, 1024),
+                 idesc_pv, (j > 0 || kk > 0));
+        mma_commit(&s.pv_done);
+        mma_commit(&s.v_empty[st]);
+        if (j + 2 < n_kv && !issue_s(j + 2)) break;
+      }
+      // TMEM must be quiescent before it is released
+      mma_commit(&s.drain);
+      mbar_wait_drain(&s.drain, 0, p.wait_limit);
+    }
+  } else {
+    // ===================================================== softmax warpgroup
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const int i = m0 + r;                 // row inside its sequence
+    const bool row_ok = i < len_q;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const float* brow = nullptr;
+    if constexpr (HAS_BIAS) {
+      if (row_ok) brow = p.bias + bidx * p.bias_bstride + ((long long)h * p.Nq + i) * p.Nk;
+    }
+    float m = -INFINITY, l = 0.f;
+    bool ok = true;
+    for (int j = 0; j < n_kv; ++j) {
+      const int buf = j & 1;
+      ok = __all_sync(0xffffffffu, mbar_wait(&s.s_full[buf], (j >> 1) & 1, ab));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t sr[4][32];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_off + kColS + buf * BN + c * 32, sr[c]);
+      tmem_wait_ld();
+#pragma unroll
+      for (int c = 0; c < 4; ++c) reg_fence(sr[c]);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.s_free[buf]);
+
+      // scale (+ bias) in log2 units, mask, row max of the block
+      const int kbase = j * BN;
+      const bool need_mask = (kbase + BN > len_k) || (p.causal && kbase + BN - 1 > m0 + diag);
+      float t[BN];
+      float mb = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < BN; ++c) {
+        float x = __uint_as_float(sr[c >> 5][c & 31]) * p.scale_log2;
+        if constexpr (HAS_BIAS) {
+          if (brow != nullptr && kbase + c < len_k) x = fmaf(__ldg(brow + kbase + c), kLog2e, x);
+        }
+        if (need_mask) {
+          const int key = kbase + c;
+          if (key >= len_k || (p.causal && key > i + diag)) x = -INFINITY;
+        }
+        t[c] = x;
+        mb = fmaxf(mb, x);
+      }
+      const float m_new = fmaxf(m, mb);
+      const float m_use = m_new == -INFINITY ? 0.f : m_new;
+      const float alpha = ex2(m - m_use);
+      float rowsum = 0.f;
+      uint32_t pk[2][32];
+#pragma unroll
+      for (int c = 0; c < BN / 2; ++c) {
+        const float p0 = ex2(t[2 * c] - m_use), p1 = ex2(t[2 * c + 1] - m_use);
+        rowsum += p0 + p1;
+        pk[c >> 5][c & 31] = pack_bf16(p0, p1);
+      }
+      l = l * alpha + rowsum;
+      // P buffer `buf` was last read by P V_{j-2}, which completed before the
+      // previous iteration's pv_done wait returned.
+      tmem_st32(tmem + lane_off + kColP + buf * 64, pk[0]);
+      tmem_st32(tmem + lane_off + kColP + buf * 64 + 32, pk[1]);
+      if (j > 0) {
+        ok = __all_sync(0xffffffffu, mbar_wait(&s.pv_done, (j - 1) & 1, ab));
+        if (!ok) break;
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t orr[32];
+            tmem_ld32(tmem + lane_off + kColO + c * 32, orr);
+            tmem_wait_ld();
+            reg_fence(orr);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) orr[e] = __float_as_uint(__uint_as_float(orr[e]) * alpha);
+            tmem_st32(tmem + lane_off + kColO + c * 32, orr);
+          }
+        }
+      }
+      m = m_new;
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.p_full[buf]);
+    }
+    // ---- epilogue: O / l -> bf16, LSE (natural log)
+    if (ok && n_kv > 0) ok = __all_sync(0xffffffffu, mbar_wait(&s.pv_done, (n_kv - 1) & 1, ab));
+    tc_fence_after();
+    if (ok) {
+      const float inv_l = l > 0.f ? 1.f / l : 0.f;
+      __nv_bfloat16* orow = p.o + bidx * p.o_bstride + ((long long)(q_off + i) * p.Hq + h) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t orr[32];
+        if (n_kv > 0) {
+          tmem_ld32(tmem + lane_off + kColO + c * 32, orr);
+          tmem_wait_ld();
+          reg_fence(orr);
+        } else {
+#pragma unroll
+          for (int e = 0; e < 32; ++e) orr[e] = 0u;
+        }
+        uint32_t packed[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e)
+          packed[e] = pack_bf16(__uint_as_float(orr[2 * e]) * inv_l, __uint_as_float(orr[2 * e + 1]) * inv_l);
+        if (row_ok) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + c * 32);
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            dst[e] = make_uint4(packed[4 * e], packed[4 * e + 1], packed[4 * e + 2], packed[4 * e + 3]);
+        }
+      }
+      if (row_ok)
+        p.lse[bidx * p.lse_bstride + (long long)h * p.lse_hstride + q_off + i] =
+            l > 0.f ? (m + __log2f(l)) * kLn2 : -INFINITY;
+    }
+  }
+
+  // ---- teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+template <int D, bool HAS_BIAS>
+int launch_fwd_t(const TcGeom& g, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                 const FwdParams& p, cudaStream_t st) {
+  // At least half of the SM's shared memory, so that a second CTA never waits
+  // on the 512 TMEM columns this one holds.
+  const size_t smem = std::max<size_t>(sizeof(FwdSmem<D>) + 1024, 116 * 1024);
+  auto kern = fwd_sm100_kernel<D, HAS_BIAS>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  const int max_nq = g.cu_q ? g.max_nq : g.Nq;
+  dim3 grid((max_nq + BM - 1) / BM, g.Hq, g.cu_q ? g.num_seqs : g.B);
+  kern<<<grid, kThreads, smem, st>>>(mq, mk, mv, p);
+  count_launch();
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+}  // namespace
+
+int launch_fwd_sm100(const TcGeom& g, __nv_bfloat16* o, float* lse, cudaStream_t st) {
+  // 4-D views (d, head, row, batch); packed inputs are one batch of `total` rows.
+  const int B = g.cu_q ? 1 : g.B;
+  CUtensorMap mq, mk, mv;
+  const uint32_t box[4] = {64, 1, 128, 1};
+  {
+    const uint64_t dims[4] = {(uint64_t)g.D, (uint64_t)g.Hq, (uint64_t)g.Nq, (uint64_t)B};
+    const uint64_t str[3] = {(uint64_t)g.D * 2, (uint64_t)g.Hq * g.D * 2, (uint64_t)g.Nq * g.Hq * g.D * 2};
+    if (encode_tmap_bf16(&mq, g.q, 4, dims, str, box) != ATTN_OK) return ATTN_ERR_CUDA;
+  }
+  {
+    const uint64_t dims[4] = {(uint64_t)g.D, (uint64_t)g.Hkv, (uint64_t)g.Nk, (uint64_t)B};
+    const uint64_t str[3] = {(uint64_t)g.D * 2, (uint64_t)g.Hkv * g.D * 2, (uint64_t)g.Nk * g.Hkv * g.D * 2};
+    if (encode_tmap_bf16(&mk, g.k, 4, dims, str, box) != ATTN_OK) return ATTN_ERR_CUDA;
+    if (encode_tmap_bf16(&mv, g.v, 4, dims, str, box) != ATTN_OK) return ATTN_ERR_CUDA;
+  }
+  FwdParams p{};
+  p.o = o;
+  p.lse = lse;
+  p.bias = g.bias;
+  p.bias_bstride = g.bias_bstride;
+  p.cu_q = g.cu_q;
+  p.cu_k = g.cu_k;
+  p.Hq = g.Hq;
+  p.Hkv = g.Hkv;
+  p.Nq = g.Nq;
+  p.Nk = g.Nk;
+  p.o_bstride = g.cu_q ? 0 : (long long)g.Nq * g.Hq * g.D;
+  p.lse_bstride = g.cu_q ? 0 : (long long)g.Hq * g.Nq;
+  p.lse_hstride = g.Nq;  // packed: Nq is the total row count
+  p.scale_log2 = g.scale * kLog2e;
+  p.causal = g.causal;
+  p.status = device_status_ptr();
+  p.wait_limit = kWaitLimitCycles;
+  if (!p.status) return ATTN_ERR_CUDA;
+  const bool has_bias = g.bias != nullptr;
+  if (g.D == 64)
+    return has_bias ? launch_fwd_t<64, true>(g, mq, mk, mv, p, st) : launch_fwd_t<64, false>(g, mq, mk, mv, p, st);
+  return has_bias ? launch_fwd_t<128, true>(g, mq, mk, mv, p, st) : launch_fwd_t<128, false>(g, mq, mk, mv, p, st);
+}
+
+}  // namespace attn

@@ -1,0 +1,64 @@
+// Host-side interface between the C-ABI layer (attn_api.cu) and the kernels.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/attn.h"
+
+namespace attn {
+
+// Launch accounting (per host thread), read by attn_launch_count.
+void count_launch(int n = 1);
+
+// Default bound on any single in-kernel wait, in SM clock cycles (~1 s).
+constexpr long long kWaitLimitCycles = 2000000000LL;
+
+// Device address of the library's status word on the current device.
+int* device_status_ptr();
+
+// ----------------------------------------------------------------- fp32 path
+struct F32Params {
+  const float *q, *k, *v, *bias;
+  float *o, *lse;
+  const int *cu_q, *cu_k;   // packed sequences (device) or null
+  long long q_bstride, k_bstride, bias_bstride, lse_bstride, lse_hstride;
+  int Hq, Hkv, Nq, Nk, D, causal;
+  float scale;
+};
+
+int launch_fwd_f32(const F32Params& p, int num_z, int max_nq, cudaStream_t st);
+int launch_bwd_f32(const F32Params& p, const float* dout, const float* Drow, float* dq, float* dk, float* dv,
+                   int num_z, int max_nq, int max_nk, cudaStream_t st);
+template <typename T>
+int launch_rowdot(const T* o, const T* dout, float* Drow, int B, int Hq, int Nq, int D, cudaStream_t st);
+
+// ------------------------------------------------------- bf16 sm_100a path
+// Geometry common to the tensor-core kernels.  Dense inputs use batch = B and
+// per-batch lengths Nq/Nk; packed inputs use batch = 1, rows = totals, and
+// per-sequence offsets from cu_q/cu_k.
+struct TcGeom {
+  const void *q, *k, *v;
+  int B, Hq, Hkv, Nq, Nk, D;   // Nq/Nk: rows per batch element (totals when packed)
+  const int *cu_q, *cu_k;      // null for dense
+  int num_seqs, max_nq, max_nk;
+  int causal;
+  float scale;
+  const float* bias;
+  long long bias_bstride;
+};
+
+int launch_fwd_sm100(const TcGeom& g, __nv_bfloat16* o, float* lse, cudaStream_t st);
+int launch_bwd_sm100(const TcGeom& g, const __nv_bfloat16* o, const float* lse, const __nv_bfloat16* dout,
+                     __nv_bfloat16* dq, __nv_bfloat16* dk, __nv_bfloat16* dv, float* dq_acc, float* Drow,
+                     cudaStream_t st);
+int launch_fwd_naive(const TcGeom& g, __nv_bfloat16* o, float* lse, float* s_scratch, __nv_bfloat16* p_scratch,
+                     cudaStream_t st);
+
+// Tensor-map encoding (driver entry point resolved at run time).
+int encode_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
+                     const uint64_t* strides_bytes, const uint32_t* box);
+
+}  // namespace attn

@@ -1,0 +1,134 @@
+/*
+ * libattn -- exact IO-aware scaled-dot-product attention for B200 (sm_100a).
+ *
+ * Computes  O = softmax(scale * Q K^T + B) V  row by row, streaming K/V tiles
+ * past a resident Q tile and carrying the online-softmax state (running max m,
+ * normaliser l, unnormalised numerator a), rescaled by exp(m - m') whenever a
+ * tile raises the maximum; the N_q x N_k score / probability matrix never
+ * reaches device memory.  The backward keeps only the per-row log-sum-exp and
+ * recomputes P tile by tile.
+ *
+ * Sources of the operation:
+ *   - "Understanding FlashAttention Pt 1", 0.2 Notation: S = QK^T/sqrt(d) + B,
+ *     P = softmax_row(S), O = PV, with B an optional additive mask or bias;
+ *   - "Softmax does not need the matrix", section "Carry the Normalizer": the
+ *     (m, l, a) state and its rescale-and-add merge of a new key block;
+ *   - "Attention IO tiling" lesson card, The mechanism: tiles of Q/K/V staged
+ *     on chip, the score block discarded, retained row statistics plus
+ *     recomputation for the backward.
+ *
+ * Conventions shared by every entry point
+ *   Pointers: caller-owned DEVICE memory unless stated otherwise; the library
+ *     allocates nothing and keeps no state between calls except the device
+ *     status word (see attn_device_status).  16-byte alignment is required for
+ *     q, k, v, o, dq, dk, dv, dout.
+ *   Layouts (row-major, innermost last):
+ *     q, o, dout, dq : [batch, n_q, h_q, d]
+ *     k, v, dk, dv   : [batch, n_k, h_kv, d]
+ *     lse            : [batch, h_q, n_q]  fp32, natural log, -inf for a row that
+ *                      sees no key
+ *     bias           : fp32 [h_q, n_q, n_k] for batch element b at
+ *                      bias + b * bias_batch_stride (stride 0 = broadcast)
+ *   dtype: ATTN_BF16 (bf16 inputs/outputs, fp32 accumulation, sm_100a tensor
+ *     cores; d in {64, 128}) or ATTN_F32 (fp32 everywhere, CUDA cores; d in
+ *     {64, 128}).
+ *   Heads: h_q must be a multiple of h_kv; query head h reads KV head
+ *     h / (h_q / h_kv) (MHA when equal, MQA when h_kv == 1).
+ *   Causal: key j is visible from query i iff j <= i + (n_k - n_q).
+ *   Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default).
+ *   Return: ATTN_OK or a negative ATTN_ERR_* code; on an error code nothing
+ *     was launched.
+ */
+#ifndef ATTN_H
+#define ATTN_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define ATTN_BF16 0
+#define ATTN_F32 1
+
+#define ATTN_OK 0
+#define ATTN_ERR_INVALID (-1)     /* null pointer, bad size, h_q % h_kv != 0, misaligned */
+#define ATTN_ERR_UNSUPPORTED (-2) /* d not in {64,128}, bias with packed inputs, no sm_100 device */
+#define ATTN_ERR_WORKSPACE (-3)   /* workspace missing or smaller than attn_bwd_workspace_size */
+#define ATTN_ERR_CUDA (-4)        /* a CUDA runtime/driver call failed */
+#define ATTN_ERR_TIMEOUT (-5)     /* a kernel gave up a bounded wait (device status word) */
+
+/*
+ * Forward.  Writes o (same dtype as q) and lse.  bias may be NULL.
+ * scale: multiplier of Q K^T (1/sqrt(d) for the standard definition).
+ */
+int attn_fwd(const void* q, const void* k, const void* v, const float* bias,
+             long long bias_batch_stride, void* o, float* lse, int batch, int h_q, int h_kv,
+             int n_q, int n_k, int d, float scale, int causal, int dtype, void* stream);
+
+/*
+ * Bytes of device workspace attn_bwd needs: an fp32 dQ accumulator
+ * [batch, n_q, h_q, d] plus the fp32 row terms D_i = dO_i . O_i [batch, h_q, n_q]
+ * (each region 256-byte aligned).  Linear in n, never n^2.
+ */
+size_t attn_bwd_workspace_size(int batch, int h_q, int n_q, int d);
+
+/*
+ * Backward of attn_fwd.  Inputs: q, k, v, bias (same as the forward), the
+ * forward's o and lse, and the upstream gradient dout.  Outputs dq, dk, dv in
+ * the dtype and layout of q, k, v; dk/dv sum the h_q / h_kv query heads of a
+ * group.  workspace: caller-owned device buffer of at least
+ * attn_bwd_workspace_size(...) bytes (contents need not be initialised).
+ */
+int attn_bwd(const void* q, const void* k, const void* v, const float* bias,
+             long long bias_batch_stride, const void* o, const float* lse, const void* dout,
+             void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int batch,
+             int h_q, int h_kv, int n_q, int n_k, int d, float scale, int causal, int dtype,
+             void* stream);
+
+/*
+ * Packed variable-length forward.  q: [total_q, h_q, d], k/v: [total_k, h_kv, d],
+ * o like q, lse: [h_q, total_q].  cu_seqlens_q / cu_seqlens_k: DEVICE int32
+ * arrays of num_seqs + 1 non-decreasing prefix offsets starting at 0; sequence z
+ * owns rows cu[z] .. cu[z+1]-1.  max_seqlen_q / max_seqlen_k bound the lengths
+ * (they size the launch).  Causal masking applies inside each sequence.  No bias.
+ */
+int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                    const int* cu_seqlens_q, const int* cu_seqlens_k, int num_seqs,
+                    int max_seqlen_q, int max_seqlen_k, int total_q, int total_k, int h_q,
+                    int h_kv, int d, float scale, int causal, int dtype, void* stream);
+
+/*
+ * Deliberately naive materialising forward, for measurement only (the
+ * three-step "standard attention" the pages contrast with: write S to device
+ * memory, read it back for the row softmax and write P, read P for P V).
+ * s_scratch: fp32 [n_q, n_k], p_scratch: bf16 [n_q, n_k], both caller-owned
+ * device buffers reused for every (batch, head).  bf16 only, no bias.
+ */
+size_t attn_naive_scratch_size(int n_q, int n_k);
+int attn_fwd_naive(const void* q, const void* k, const void* v, void* o, float* lse,
+                   void* scratch, size_t scratch_bytes, int batch, int h_q, int h_kv, int n_q,
+                   int n_k, int d, float scale, int causal, void* stream);
+
+/* Human-readable text for an ATTN_* code (static storage). */
+const char* attn_strerror(int code);
+
+/*
+ * Synchronises `stream`, then returns and clears the device status word of the
+ * current device: ATTN_OK, or ATTN_ERR_TIMEOUT if a kernel launched since the
+ * last call abandoned a bounded wait (its outputs are then undefined).
+ */
+int attn_device_status(void* stream);
+
+/*
+ * Kernel launches issued by this library on the calling host thread since the
+ * last reset (reset = 1 clears after reading).  Lets callers count the GPU
+ * work of a timed region.
+ */
+long long attn_launch_count(int reset);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* ATTN_H */
