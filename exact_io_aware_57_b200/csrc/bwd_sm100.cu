@@ -1,8 +1,503 @@
+// Backward attention on sm_100a tensor cores: recompute P tile by tile from
+// the stored per-row log-sum-exp ("Attention IO tiling" lesson card, The
+// mechanism: use the retained statistics and permitted recomputation for
+// backward execution; "Understanding FlashAttention Pt 1", 3.6 backward pass:
+// recompute instead of save).  The pages print no gradient formulas; the
+// kernel forms the exact gradient of softmax(scale QK^T + B)V:
+//   P = exp(scale S + B - LSE),  dV = P^T dO,  dP = dO V^T,
+//   dS = P o (dP - D) with D_i = dO_i . O_i,  dQ = scale dS K,  dK = scale dS^T Q.
+//
+// Three launches:
+//   bwd_pre    D_i = dO_i . O_i (fp32) and zero the fp32 dQ accumulator
+//   bwd_main   one CTA per (128-key tile, KV head, batch); K_j and V_j stay in
+//              shared memory, dK_j and dV_j accumulate in TMEM over every query
+//              tile and every query head of the group
+//   bwd_dq     dQ = scale * accumulator -> bf16
+//
+// bwd_main roles (10 warps):
+//   warp 0      TMA producer (K_j, V_j once; Q_i, dO_i per step) + LSE/D rows
+//   warp 1      TMEM owner + single-thread tcgen05.mma issuer
+//   warps 2..5  thread t owns key row t: P^T, dS^T, and the dK/dV epilogue
+//   warps 6..9  thread t owns query row t of the dQ tile: TMEM -> fp32 reductions
+// TMEM columns: [0,128) S^T (then P^T as bf16 pairs in [0,64)),
+//   [128,256) dP^T (then the dQ tile), [256,256+D) dV, [256+D,256+2D) dK.
+// Per step (query head h, query tile i):
+//   MMA   S^T = K_j Q_i^T,  dP^T = V_j dO_i^T
+//   WG0   P^T = 2^(scale log2e S^T + log2e B^T - log2e LSE) -> TMEM (bf16);
+//         dS^T = P^T o (dP^T - D) -> shared memory (bf16, 128B-swizzled)
+//   MMA   dV += P^T dO_i (P^T from TMEM), dK += dS^T Q_i, dQ_i = dS K_j
+//   WG1   dQ_i -> red.global.add into the fp32 accumulator
+#include <algorithm>
+
 #include "common.cuh"
 #include "kernels.h"
+
 namespace attn {
-int launch_bwd_sm100(const TcGeom&, const __nv_bfloat16*, const float*, const __nv_bfloat16*, __nv_bfloat16*,
-                     __nv_bfloat16*, __nv_bfloat16*, float*, float*, cudaStream_t) {
-  return ATTN_ERR_UNSUPPORTED;
+
+namespace {
+
+constexpr int BM = 128;   // query rows per step
+constexpr int BN = 128;   // keys per CTA
+constexpr int NSTQ = 2;   // Q/dO stages
+constexpr int kThreads = 320;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kColST = 0, kColDPT = 128, kColDV = 256;
+
+template <int D>
+struct BwdSmem {
+  static constexpr int kTileBytes = 128 * D * 2;
+  alignas(1024) uint8_t k[kTileBytes];
+  alignas(1024) uint8_t v[kTileBytes];
+  alignas(1024) uint8_t q[NSTQ][kTileBytes];
+  alignas(1024) uint8_t dout[NSTQ][kTileBytes];
+  alignas(1024) uint8_t ds[128 * 128 * 2];  // dS^T, [key][query] in two 64-column blocks
+  float lse2[NSTQ][BM];                     // log2(e) * LSE of the step's query rows (+inf: no key)
+  float drow[NSTQ][BM];                     // D_i of the step's query rows
+  uint64_t kv_full, q_full[NSTQ], q_empty[NSTQ];
+  uint64_t s_full, ds_ready, dq_full, dq_drained, drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+struct BwdParams {
+  const float* lse;
+  const float* drow;
+  float* dq_acc;
+  __nv_bfloat16* dk;
+  __nv_bfloat16* dv;
+  const float* bias;
+  long long bias_bstride;
+  int Hq, Hkv, Nq, Nk;
+  float scale, scale_log2;
+  int causal;
+  int* status;
+  long long wait_limit;
+};
+
+template <int N>
+ATTN_DEVINL void reg_fence(uint32_t (&r)[N]) {
+#pragma unroll
+  for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
 }
+
+ATTN_DEVINL void red_add_v4(float* addr, float a, float b, float c, float d) {
+  asm volatile("red.relaxed.gpu.global.add.v4.f32 [%0], {%1,%2,%3,%4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
+
+ATTN_DEVINL void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
+template <int D, bool HAS_BIAS>
+__global__ void __launch_bounds__(kThreads, 1)
+    bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                    const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                    const BwdParams p) {
+  using Smem = BwdSmem<D>;
+  constexpr int KB = D / 64;
+  constexpr uint32_t kColDK = kColDV + D;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  Smem& s = *reinterpret_cast<Smem*>(smem_raw);
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  const int n_tile = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
+  const int n0 = n_tile * BN;
+  const int len_q = p.Nq, len_k = p.Nk;
+  const int diag = len_k - len_q;  // key j visible from query i iff j <= i + diag
+  const int G = p.Hq / p.Hkv;
+  const int n_qt = (len_q + BM - 1) / BM;
+  int i_first = 0;
+  if (p.causal) {
+    const int first_row = n0 - diag;  // first query row that sees key n0
+    i_first = first_row <= 0 ? 0 : first_row / BM;
+  }
+  const int per_head = i_first < n_qt ? n_qt - i_first : 0;
+  const int n_steps = G * per_head;
+
+  if ((smem_u32(smem_raw) & 1023u) != 0) {  // the swizzle needs 1024-byte aligned tiles
+    if (threadIdx.x == 0) atomicExch(p.status, ATTN_ERR_CUDA);
+    return;
+  }
+  if (threadIdx.x == 0) {
+    s.abort_flag = 0;
+    mbar_init(&s.kv_full, 1);
+    for (int i = 0; i < NSTQ; ++i) {
+      mbar_init(&s.q_full[i], 1 + 32);  // TMA transaction arrive + 32 producer lanes (LSE/D rows)
+      mbar_init(&s.q_empty[i], 1);
+    }
+    mbar_init(&s.s_full, 1);
+    mbar_init(&s.ds_ready, 4);
+    mbar_init(&s.dq_full, 1);
+    mbar_init(&s.dq_drained, 4);
+    mbar_init(&s.drain, 1);
+    fence_mbar_init();
+  }
+  if (warp == 1) tmem_alloc(&s.tmem_base, kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = s.tmem_base;
+  const Abort ab{&s.abort_flag, p.status, p.wait_limit};
+
+  if (warp == 0) {
+    // ===================================================== producer
+    int issued = 0;
+    if (lane == 0) {
+      tma_prefetch_desc(&tm_q);
+      tma_prefetch_desc(&tm_k);
+      tma_prefetch_desc(&tm_v);
+      tma_prefetch_desc(&tm_do);
+      if (n_steps > 0) {
+        mbar_expect_tx(&s.kv_full, 2 * Smem::kTileBytes);
+#pragma unroll
+        for (int kb = 0; kb < KB; ++kb) {
+          tma_load_4d(s.k + kb * BN * 128, &tm_k, &s.kv_full, kb * 64, hk, n0, b);
+          tma_load_4d(s.v + kb * BN * 128, &tm_v, &s.kv_full, kb * 64, hk, n0, b);
+        }
+      }
+    }
+    for (int step = 0; step < n_steps; ++step) {
+      const int st = step % NSTQ;
+      const uint32_t ph = (step / NSTQ) & 1;
+      const int h = hk * G + step / per_head;
+      const int i0 = (i_first + step % per_head) * BM;
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(&s.q_empty[st], ph ^ 1, ab));
+      if (!ok) break;
+      if (lane == 0) {
+        mbar_expect_tx(&s.q_full[st], 2 * Smem::kTileBytes);
+#pragma unroll
+        for (int kb = 0; kb < KB; ++kb) {
+          tma_load_4d(s.q[st] + kb * BM * 128, &tm_q, &s.q_full[st], kb * 64, h, i0, b);
+          tma_load_4d(s.dout[st] + kb * BM * 128, &tm_do, &s.q_full[st], kb * 64, h, i0, b);
+        }
+      }
+      const long long row0 = ((long long)b * p.Hq + h) * p.Nq;
+#pragma unroll
+      for (int e = 0; e < BM / 32; ++e) {
+        const int c = lane + 32 * e;
+        const int qi = i0 + c;
+        float l2 = INFINITY, dr = 0.f;
+        if (qi < len_q) {
+          const float lse = p.lse[row0 + qi];
+          l2 = lse == -INFINITY ? INFINITY : lse * kLog2e;
+          dr = p.drow[row0 + qi];
+        }
+        s.lse2[st][c] = l2;
+        s.drow[st][c] = dr;
+      }
+      mbar_arrive(&s.q_full[st]);
+      ++issued;
+    }
+    if (lane == 0 && s.abort_flag) {
+      if (n_steps > 0) mbar_wait_drain(&s.kv_full, 0, p.wait_limit);
+      for (int j = max(0, issued - NSTQ); j < issued; ++j)
+        mbar_wait_drain(&s.q_full[j % NSTQ], (j / NSTQ) & 1, p.wait_limit);
+    }
+  } else if (warp == 1) {
+    // ===================================================== MMA issuer
+    if (lane == 0 && n_steps > 0) {
+      constexpr uint32_t idesc_s = idesc_bf16(BN, BM, 0, 0);    // K_j / V_j (K-major) x Q_i / dO_i (K-major)
+      constexpr uint32_t idesc_kv = idesc_bf16(BN, D, 0, 1);    // P^T, dS^T (K-major) x dO_i / Q_i (MN-major)
+      constexpr uint32_t idesc_dq = idesc_bf16(BM, D, 1, 1);    // dS (MN-major) x K_j (MN-major)
+      const uint32_t k_addr = smem_u32(s.k), v_addr = smem_u32(s.v), ds_addr = smem_u32(s.ds);
+      bool ok = mbar_wait(&s.kv_full, 0, ab);
+      for (int step = 0; ok && step < n_steps; ++step) {
+        const int st = step % NSTQ;
+        if (!mbar_wait(&s.q_full[st], (step / NSTQ) & 1, ab)) break;
+        // dQ of the previous step must have left TMEM (it lives where dP^T goes)
+        if (step > 0 && !mbar_wait(&s.dq_drained, (step - 1) & 1, ab)) break;
+        tc_fence_after();
+        const uint32_t q_addr = smem_u32(s.q[st]), do_addr = smem_u32(s.dout[st]);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+          mma_ss(tmem + kColST, sdesc_sw128(k_addr + off, 16, 1024), sdesc_sw128(q_addr + off, 16, 1024), idesc_s,
+                 kk > 0);
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+          mma_ss(tmem + kColDPT, sdesc_sw128(v_addr + off, 16, 1024), sdesc_sw128(do_addr + off, 16, 1024),
+                 idesc_s, kk > 0);
+        }
+        mma_commit(&s.s_full);
+        if (!mbar_wait(&s.ds_ready, step & 1, ab)) break;
+        tc_fence_after();
+        // dV += P^T dO_i   (A: P^T bf16 in TMEM, K = query)
+#pragma unroll
+        for (int kk = 0; kk < BM / 16; ++kk)
+          mma_ts(tmem + kColDV, tmem + kColST + kk * 8, sdesc_sw128(do_addr + kk * 2048, BM * 128, 1024), idesc_kv,
+                 (step > 0 || kk > 0));
+        // dK += dS^T Q_i  (A: dS^T in shared memory, K-major over queries)
+#pragma unroll
+        for (int kk = 0; kk < BM / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+          mma_ss(tmem + kColDK, sdesc_sw128(ds_addr + off, 16, 1024), sdesc_sw128(q_addr + kk * 2048, BM * 128, 1024),
+                 idesc_kv, (step > 0 || kk > 0));
+        }
+        mma_commit(&s.q_empty[st]);
+        // dQ_i = dS K_j  (A: the same dS^T buffer read MN-major, K = key)
+#pragma unroll
+        for (int kk = 0; kk < BN / 16; ++kk)
+          mma_ss(tmem + kColDPT, sdesc_sw128(ds_addr + kk * 2048, 128 * 128, 1024),
+                 sdesc_sw128(k_addr + kk * 2048, BN * 128, 1024), idesc_dq, kk > 0);
+        mma_commit(&s.dq_full);
+      }
+      mma_commit(&s.drain);
+      mbar_wait_drain(&s.drain, 0, p.wait_limit);
+    }
+  } else if (warp < 6) {
+    // ===================================================== P^T / dS^T (thread = key row)
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const int kj = n0 + r;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const uint32_t ds_row = smem_u32(s.ds) + r * 128;
+    bool ok = true;
+    for (int step = 0; step < n_steps; ++step) {
+      const int st = step % NSTQ;
+      const int h = hk * G + step / per_head;
+      const int i0 = (i_first + step % per_head) * BM;
+      ok = __all_sync(0xffffffffu, mbar_wait(&s.s_full, step & 1, ab));
+      if (!ok) break;
+      // q_full for this stage completed before s_full (the MMA waited on it)
+      tc_fence_after();
+      const bool need_mask = (kj >= len_k) || (i0 + BM > len_q) || (p.causal && n0 + BN - 1 > i0 + diag);
+      const float* bcol = nullptr;
+      if constexpr (HAS_BIAS) {
+        if (kj < len_k) bcol = p.bias + b * p.bias_bstride + (long long)h * p.Nq * p.Nk + kj;
+      }
+#pragma unroll
+      for (int c = 0; c < BM / 32; ++c) {
+        uint32_t sr[32], dpr[32];
+        tmem_ld32(tmem + lane_off + kColST + c * 32, sr);
+        tmem_ld32(tmem + lane_off + kColDPT + c * 32, dpr);
+        tmem_wait_ld();
+        reg_fence(sr);
+        reg_fence(dpr);
+        uint32_t pk[16], dk[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          float pv[2], dsv[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int col = c * 32 + e + u;
+            const int qi = i0 + col;
+            float t = __uint_as_float(sr[e + u]) * p.scale_log2 - s.lse2[st][col];
+            if constexpr (HAS_BIAS) {
+              if (bcol != nullptr && qi < len_q) t = fmaf(__ldg(bcol + (long long)qi * p.Nk), kLog2e, t);
+            }
+            float pe = ex2(t);
+            if (need_mask && (kj >= len_k || qi >= len_q || (p.causal && kj > qi + diag))) pe = 0.f;
+            pv[u] = pe;
+            dsv[u] = pe * (__uint_as_float(dpr[e + u]) - s.drow[st][col]);
+          }
+          pk[e >> 1] = pack_bf16(pv[0], pv[1]);
+          dk[e >> 1] = pack_bf16(dsv[0], dsv[1]);
+        }
+        // P^T columns [16c, 16c+16) lie in S^T columns already read
+        tmem_st16(tmem + lane_off + kColST + c * 16, pk);
+        // dS^T: 32 queries = 4 chunks of 16 bytes in 64-column block c/2
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int chunk = (c & 1) * 4 + u;  // 16-byte chunk within the 128-byte row
+          const uint32_t addr = ds_row + (c >> 1) * (128 * 128) + ((chunk ^ (r & 7)) << 4);
+          st_shared_v4(addr, dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
+        }
+      }
+      tmem_wait_st();
+      fence_proxy_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.ds_ready);
+    }
+    // ---- epilogue: dK (scaled) and dV for this thread's key row
+    if (ok && n_steps > 0) ok = __all_sync(0xffffffffu, mbar_wait(&s.dq_full, (n_steps - 1) & 1, ab));
+    tc_fence_after();
+    if (ok) {
+      const long long row = (((long long)b * p.Nk + kj) * p.Hkv + hk) * D;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const uint32_t col0 = half == 0 ? kColDV : kColDK;
+        const float mul = half == 0 ? 1.f : p.scale;
+        __nv_bfloat16* dst = (half == 0 ? p.dv : p.dk) + row;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c) {
+          uint32_t a[32];
+          if (n_steps > 0) {
+            tmem_ld32(tmem + lane_off + col0 + c * 32, a);
+            tmem_wait_ld();
+            reg_fence(a);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) a[e] = 0u;
+          }
+          uint32_t pkd[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e)
+            pkd[e] = pack_bf16(__uint_as_float(a[2 * e]) * mul, __uint_as_float(a[2 * e + 1]) * mul);
+          if (kj < len_k) {
+            uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) d4[e] = make_uint4(pkd[4 * e], pkd[4 * e + 1], pkd[4 * e + 2], pkd[4 * e + 3]);
+          }
+        }
+      }
+    }
+  } else {
+    // ===================================================== dQ drain (thread = query row)
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    for (int step = 0; step < n_steps; ++step) {
+      const int h = hk * G + step / per_head;
+      const int qi = (i_first + step % per_head) * BM + r;
+      if (!__all_sync(0xffffffffu, mbar_wait(&s.dq_full, step & 1, ab))) break;
+      tc_fence_after();
+      float* dst = p.dq_acc + (((long long)b * p.Nq + qi) * p.Hq + h) * D;
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) {
+        uint32_t a[32];
+        tmem_ld32(tmem + lane_off + kColDPT + c * 32, a);
+        tmem_wait_ld();
+        reg_fence(a);
+        if (qi < len_q) {
+#pragma unroll
+          for (int e = 0; e < 32; e += 4)
+            red_add_v4(dst + c * 32 + e, __uint_as_float(a[e]), __uint_as_float(a[e + 1]), __uint_as_float(a[e + 2]),
+                       __uint_as_float(a[e + 3]));
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.dq_drained);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+// D_i = dO_i . O_i (fp32) and zeroed dQ accumulator rows.  One warp per (b, n, h) row.
+template <int D>
+__global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16* __restrict__ o,
+                                                      const __nv_bfloat16* __restrict__ dout, float* __restrict__ drow,
+                                                      float* __restrict__ dq_acc, int B, int Hq, int Nq) {
+  constexpr int E = D / 32;  // bf16 per lane (2 or 4)
+  const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (row >= (long long)B * Nq * Hq) return;
+  float acc = 0.f;
+  const __nv_bfloat16* orow = o + row * D + lane * E;
+  const __nv_bfloat16* drw = dout + row * D + lane * E;
+#pragma unroll
+  for (int e = 0; e < E; ++e) acc = fmaf(__bfloat162float(orow[e]), __bfloat162float(drw[e]), acc);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  float* q = dq_acc + row * D + lane * E;
+#pragma unroll
+  for (int e = 0; e < E; ++e) q[e] = 0.f;
+  if (lane == 0) {
+    const int h = (int)(row % Hq);
+    const long long bn = row / Hq;
+    const int n = (int)(bn % Nq), bb = (int)(bn / Nq);
+    drow[((long long)bb * Hq + h) * Nq + n] = acc;
+  }
+}
+
+// dQ = scale * accumulator, fp32 -> bf16, 8 elements per thread.
+__global__ void __launch_bounds__(256) bwd_dq_kernel(const float* __restrict__ acc, __nv_bfloat16* __restrict__ dq,
+                                                     long long n8, float scale) {
+  const long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n8) return;
+  const float4 a = reinterpret_cast<const float4*>(acc)[2 * i];
+  const float4 c = reinterpret_cast<const float4*>(acc)[2 * i + 1];
+  reinterpret_cast<uint4*>(dq)[i] = make_uint4(pack_bf16(a.x * scale, a.y * scale), pack_bf16(a.z * scale, a.w * scale),
+                                               pack_bf16(c.x * scale, c.y * scale), pack_bf16(c.z * scale, c.w * scale));
+}
+
+template <int D, bool HAS_BIAS>
+int launch_main_t(const TcGeom& g, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                  const CUtensorMap& mdo, const BwdParams& p, cudaStream_t st) {
+  const size_t smem = std::max<size_t>(sizeof(BwdSmem<D>), 116 * 1024);
+  auto kern = bwd_main_kernel<D, HAS_BIAS>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
+    return ATTN_ERR_CUDA;
+  dim3 grid((g.Nk + BN - 1) / BN, g.Hkv, g.B);
+  kern<<<grid, kThreads, smem, st>>>(mq, mk, mv, mdo, p);
+  count_launch();
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
+}  // namespace
+
+int launch_bwd_sm100(const TcGeom& g, const __nv_bfloat16* o, const float* lse, const __nv_bfloat16* dout,
+                     __nv_bfloat16* dq, __nv_bfloat16* dk, __nv_bfloat16* dv, float* dq_acc, float* Drow,
+                     cudaStream_t st) {
+  if (g.cu_q) return ATTN_ERR_UNSUPPORTED;
+  // 1) D and zeroed accumulator
+  {
+    const long long rows = (long long)g.B * g.Nq * g.Hq;
+    const unsigned blocks = (unsigned)((rows + 7) / 8);
+    if (g.D == 64)
+      bwd_pre_kernel<64><<<blocks, 256, 0, st>>>(o, dout, Drow, dq_acc, g.B, g.Hq, g.Nq);
+    else
+      bwd_pre_kernel<128><<<blocks, 256, 0, st>>>(o, dout, Drow, dq_acc, g.B, g.Hq, g.Nq);
+    count_launch();
+    if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
+  }
+  // 2) main
+  CUtensorMap mq, mk, mv, mdo;
+  const uint32_t box[4] = {64, 1, 128, 1};
+  {
+    const uint64_t dims[4] = {(uint64_t)g.D, (uint64_t)g.Hq, (uint64_t)g.Nq, (uint64_t)g.B};
+    const uint64_t str[3] = {(uint64_t)g.D * 2, (uint64_t)g.Hq * g.D * 2, (uint64_t)g.Nq * g.Hq * g.D * 2};
+    if (encode_tmap_bf16(&mq, g.q, 4, dims, str, box) != ATTN_OK) return ATTN_ERR_CUDA;
+    if (encode_tmap_bf16(&mdo, dout, 4, dims, str, box) != ATTN_OK) return ATTN_ERR_CUDA;
+  }
+  {
+    const uint64_t dims[4] = {(uint64_t)g.D, (uint64_t)g.Hkv, (uint64_t)g.Nk, (uint64_t)g.B};
+    const uint64_t str[3] = {(uint64_t)g.D * 2, (uint64_t)g.Hkv * g.D * 2, (uint64_t)g.Nk * g.Hkv * g.D * 2};
+    if (encode_tmap_bf16(&mk, g.k, 4, dims, str, box) != ATTN_OK) return ATTN_ERR_CUDA;
+    if (encode_tmap_bf16(&mv, g.v, 4, dims, str, box) != ATTN_OK) return ATTN_ERR_CUDA;
+  }
+  BwdParams p{};
+  p.lse = lse;
+  p.drow = Drow;
+  p.dq_acc = dq_acc;
+  p.dk = dk;
+  p.dv = dv;
+  p.bias = g.bias;
+  p.bias_bstride = g.bias_bstride;
+  p.Hq = g.Hq;
+  p.Hkv = g.Hkv;
+  p.Nq = g.Nq;
+  p.Nk = g.Nk;
+  p.scale = g.scale;
+  p.scale_log2 = g.scale * kLog2e;
+  p.causal = g.causal;
+  p.status = device_status_ptr();
+  p.wait_limit = kWaitLimitCycles;
+  if (!p.status) return ATTN_ERR_CUDA;
+  int rc;
+  const bool hb = g.bias != nullptr;
+  if (g.D == 64)
+    rc = hb ? launch_main_t<64, true>(g, mq, mk, mv, mdo, p, st) : launch_main_t<64, false>(g, mq, mk, mv, mdo, p, st);
+  else
+    rc = hb ? launch_main_t<128, true>(g, mq, mk, mv, mdo, p, st)
+            : launch_main_t<128, false>(g, mq, mk, mv, mdo, p, st);
+  if (rc) return rc;
+  // 3) dQ
+  const long long n8 = (long long)g.B * g.Nq * g.Hq * g.D / 8;
+  bwd_dq_kernel<<<(unsigned)((n8 + 255) / 256), 256, 0, st>>>(dq_acc, dq, n8, g.scale);
+  count_launch();
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
+}
+
 }  // namespace attn

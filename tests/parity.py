@@ -104,3 +104,37 @@ def check_fwd_sampled(orc, q, k, v, o, lse, causal, heads, rows, bias_fn=None, s
         worst_o = max(worst_o, max_abs(o[b, rows, h].double().numpy(), o_ref))
         worst_l = max(worst_l, max_abs(lse[b, h, rows].double().numpy(), l_ref))
     return worst_o, worst_l
+
+
+def gpu_fwd_bwd(inp, causal, bias=None, scale=None):
+    """Forward then backward through the C-ABI on cuda:0; returns CPU tensors."""
+    from exact_io_aware_57_b200 import attn
+
+    q, k, v, do = (t.cuda() for t in (inp.q, inp.k, inp.v, inp.dout))
+    bd = None if bias is None else bias.cuda()
+    o, lse = attn.attn_fwd(q, k, v, bias=bd, causal=causal, scale=scale)
+    bufs = [guarded_empty(t.shape, t.dtype) for t in (q, k, v)]
+    dq, dk, dv = attn.attn_bwd(q, k, v, o, lse, do, bias=bd, causal=causal, scale=scale,
+                               dq=bufs[0][1], dk=bufs[1][1], dv=bufs[2][1])
+    torch.cuda.synchronize()
+    assert attn.attn_device_status() == 0
+    assert all(guards_intact(b[0]) for b in bufs), "backward wrote outside its outputs"
+    return o.cpu(), lse.cpu(), dq.cpu(), dk.cpu(), dv.cpu()
+
+
+def check_bwd(orc, B, Hq, Hkv, Nq, Nk, d, causal, *, dtype=torch.bfloat16, sigma=1.0, bias=False, seed=0):
+    inp = synth.make_dense(B, Hq, Hkv, Nq, Nk, d, dtype=dtype, seed=seed, sigma_qk=sigma)
+    b = synth.alibi_like_bias(Hq, Nq, Nk) if bias else None
+    o, lse, dq, dk, dv = gpu_fwd_bwd(inp, causal, bias=b)
+    o_ref, _ = orc.fwd(inp.q, inp.k, inp.v, bias=b, causal=causal)
+    dq_r, dk_r, dv_r = orc.bwd(inp.q, inp.k, inp.v, inp.dout, bias=b, causal=causal)
+    errs = {}
+    if dtype == torch.float32:
+        for name, a, r in (("o", o, o_ref), ("dq", dq, dq_r), ("dk", dk, dk_r), ("dv", dv, dv_r)):
+            errs[name] = max_abs(a.double().numpy(), r)
+            assert errs[name] <= TOL_F32, f"{name} max-abs {errs[name]:.3e} > {TOL_F32}"
+    else:
+        for name, a, r in (("dq", dq, dq_r), ("dk", dk, dk_r), ("dv", dv, dv_r)):
+            errs[name] = rel_fro(a.double().numpy(), r)
+            assert errs[name] <= TOL_GRAD_BF16, f"{name} rel Frobenius {errs[name]:.3e} > {TOL_GRAD_BF16}"
+    return errs
