@@ -1,0 +1,398 @@
+#!/usr/bin/env python3
+"""Benchmark of the exact IO-aware attention hot path on B200.
+
+One step = the whole path once: forward (O, LSE) then backward (dQ, dK, dV)
+of causal bf16 attention, batch 2, 32 heads, N = 8192, d = 128, Q/K ~ N(0, 3^2),
+V/dO ~ N(0, 1) (seeded synthetic inputs; no dataset is involved).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+N > 1 is launched with torchrun, one process per GPU: every rank runs its own
+independent problem of the same shape (weak scaling, no collective on the data
+path); the timed region is bracketed by a barrier + device synchronisation and
+the max over ranks is reported.  Rank 0 prints one JSON line.
+
+``--impl reference`` times the fp64 CPU oracle on the host cores instead (a
+bounded causal-prefix sample of the same workload per step).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+from pathlib import Path
+
+ROOT = Path(__file__).resolve().parent
+sys.path.insert(0, str(ROOT))
+
+METRIC = "attention fwd / fwd+bwd TFLOP/s, causal bf16 N=8192 d=128; % of BF16 peak"
+SPEC_BF16_TFLOPS = 2250.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+TRAFFIC_FILE = ROOT / "profiles" / "bwd_main_causal_b2h32n8192d128_traffic.txt"
+BWD_SOURCE = ROOT / "exact_io_aware_57_b200" / "csrc" / "bwd_sm100.cu"
+
+
+# ------------------------------------------------------------------ plumbing
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=100)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
+    ap.add_argument("--no-cpu-baseline", action="store_true", help="skip timing the CPU oracle")
+    ap.add_argument("--batch", type=int, default=None, help="override the batch (profiling a smaller case)")
+    ap.add_argument("--heads", type=int, default=None, help="override the head count (profiling a smaller case)")
+    return ap.parse_args(argv)
+
+
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+def init_dist(world: int, backend: str):
+    import datetime
+
+    import torch.distributed as dist
+
+    if world > 1 and not dist.is_initialized():
+        dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist if world > 1 else None
+
+
+def barrier(dist, device=None):
+    if dist is not None:
+        if device is not None:
+            dist.barrier(device_ids=[device])
+        else:
+            dist.barrier()
+
+
+def max_over_ranks(dist, x: float, device=None) -> float:
+    """Max of a per-rank float over all ranks (identity on one process)."""
+    if dist is None:
+        return float(x)
+    import torch
+
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device if device is not None else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_seed(seed: int, rank: int) -> int:
+    """Each rank draws its own independent problem."""
+    return int(seed) * 1000 + int(rank)
+
+
+def measured_peaks():
+    p = ROOT / "MEASURED_PEAKS.json"
+    if p.exists():
+        d = json.loads(p.read_text())
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def source_digest(path: Path) -> str:
+    return hashlib.sha256(path.read_bytes()).hexdigest()[:16]
+
+
+def recorded_traffic():
+    """DRAM bytes per backward-main launch from the committed ncu summary, or None
+    if absent or if the kernel source changed since the counters were taken."""
+    if not TRAFFIC_FILE.exists():
+        return None
+    kv = {}
+    for line in TRAFFIC_FILE.read_text().splitlines():
+        if ":" in line and not line.startswith("#"):
+            k, v = line.split(":", 1)
+            kv[k.strip()] = v.strip()
+    if kv.get("kernel_source_sha256_16") != source_digest(BWD_SOURCE):
+        return None
+    try:
+        return int(kv["dram_bytes_per_full_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi clock/throttle samples every 200 ms while the timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = Path(tempfile.mkstemp(prefix="clocks_", suffix=".csv")[1])
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            time.sleep(0.6)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        rows = []
+        for line in self.path.read_text().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        self.path.unlink(missing_ok=True)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unsampled"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        busy = [x for x in sm if x > 0.5 * (max(mx) if mx else 1)] or sm
+        return {"sm_mhz": statistics.median(busy) if busy else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ------------------------------------------------------------ CPU oracle side
+def oracle_sample(prefix: int, heads: int, seed: int):
+    """Time the fp64 oracle on a causal prefix of `prefix` tokens of `heads`
+    heads (batch element 0) of the workload: rows 0..prefix-1 attend only to
+    keys 0..prefix-1, so this is an exact sub-problem.  Returns (seconds, flops)."""
+    import oracle
+    from exact_io_aware_57_b200 import synth, workloads
+
+    inp = synth.make_dense(1, heads, heads, prefix, prefix, 128, sigma_qk=3.0, seed=seed)
+    orc = oracle.get()
+    t0 = time.perf_counter()
+    orc.fwd(inp.q, inp.k, inp.v, causal=True)
+    orc.bwd(inp.q, inp.k, inp.v, inp.dout, causal=True)
+    dt = time.perf_counter() - t0
+    flops = workloads.fwd_flops_pair(prefix, prefix, 128, True) * heads * 3.5
+    return dt, flops
+
+
+def cpu_threads() -> int:
+    import oracle
+
+    return oracle.cpu_threads()
+
+
+def plan_oracle_sample(target_s: float):
+    """Pick (prefix, heads) so one oracle sample takes about target_s seconds:
+    one head per host thread (the oracle parallelises over heads), prefix from a
+    short calibration (cost grows as prefix^2)."""
+    heads = max(1, min(cpu_threads(), 64))
+    dt, _ = oracle_sample(256, heads, 0)
+    per = dt / (256.0 ** 2)
+    prefix = int(math.sqrt(max(target_s, 0.05) / max(per, 1e-12)))
+    prefix = max(256, min(8192, prefix // 128 * 128))
+    return prefix, heads
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args):
+    import torch
+
+    from exact_io_aware_57_b200 import attn, synth, workloads
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    dist = init_dist(world, "nccl")
+    w = workloads.WORKLOADS["c3"]
+    if args.batch or args.heads:
+        import dataclasses
+
+        w = dataclasses.replace(w, name=w.name + " (reduced for profiling)", batch=args.batch or w.batch,
+                                h_q=args.heads or w.h_q, h_kv=args.heads or w.h_kv)
+    B, H, N, d = w.batch, w.h_q, w.n, w.d
+    inp = synth.make_dense(B, H, H, N, N, d, sigma_qk=w.sigma_qk, seed=rank_seed(args.seed, rank))
+    host = {n: getattr(inp, n).pin_memory() for n in ("q", "k", "v", "dout")}
+    q, k, v, do = (host[n].to(dev) for n in ("q", "k", "v", "dout"))
+    o = torch.empty_like(q)
+    lse = torch.empty((B, H, N), device=dev, dtype=torch.float32)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws = torch.empty(attn.attn_bwd_workspace_size(B, H, N, d), device=dev, dtype=torch.uint8)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        attn.attn_fwd(q, k, v, causal=True, out=o, lse=lse)
+        attn.attn_bwd(q, k, v, o, lse, do, causal=True, workspace=ws, dq=dq, dk=dk, dv=dv)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if attn.attn_device_status() != 0:
+        raise RuntimeError("device status reported a timeout during warm-up")
+
+    K = args.steps
+    fwd_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    bwd_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for a, b in fwd_ev + bwd_ev:  # torch creates the CUDA event on its first record
+        a.record(stream)
+        b.record(stream)
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    clocks.start()
+    barrier(dist, local)
+    torch.cuda.synchronize()
+    attn.attn_launch_count(reset=True)
+    t_start.record(stream)
+    for i in range(K):
+        attn.attn_set_kernel_events(attn.ATTN_KERNEL_FWD, *fwd_ev[i])
+        attn.attn_set_kernel_events(attn.ATTN_KERNEL_BWD, *bwd_ev[i])
+        step()
+    t_end.record(stream)
+    torch.cuda.synchronize()
+    launches = attn.attn_launch_count(reset=True)
+    barrier(dist, local)
+    clk = clocks.stop()
+    attn.attn_set_kernel_events(attn.ATTN_KERNEL_FWD)
+    attn.attn_set_kernel_events(attn.ATTN_KERNEL_BWD)
+    if attn.attn_device_status() != 0:
+        raise RuntimeError("device status reported a timeout in the timed region")
+
+    ms_total = max_over_ranks(dist, t_start.elapsed_time(t_end), dev)
+    ms_step = ms_total / K
+    fwd_ms = statistics.mean(a.elapsed_time(b) for a, b in fwd_ev)
+    bwd_main_ms = statistics.mean(a.elapsed_time(b) for a, b in bwd_ev)
+    fwd_ms = max_over_ranks(dist, fwd_ms, dev)
+    bwd_main_ms = max_over_ranks(dist, bwd_main_ms, dev)
+    f_fwd = workloads.flops(w, backward=False)
+    f_step = workloads.flops(w, backward=True)
+    value = world * f_step / (ms_step * 1e-3) / 1e12
+
+    # ---- end to end through the public API with pinned host buffers
+    e2e = None
+    if not args.no_e2e:
+        out_host = {"o": torch.empty_like(host["q"]).pin_memory(), "lse": torch.empty((B, H, N)).pin_memory(),
+                    "dq": torch.empty_like(host["q"]).pin_memory(), "dk": torch.empty_like(host["k"]).pin_memory(),
+                    "dv": torch.empty_like(host["v"]).pin_memory()}
+
+        def e2e_step():
+            q.copy_(host["q"], non_blocking=True)
+            k.copy_(host["k"], non_blocking=True)
+            v.copy_(host["v"], non_blocking=True)
+            do.copy_(host["dout"], non_blocking=True)
+            step()
+            out_host["o"].copy_(o, non_blocking=True)
+            out_host["lse"].copy_(lse, non_blocking=True)
+            out_host["dq"].copy_(dq, non_blocking=True)
+            out_host["dk"].copy_(dk, non_blocking=True)
+            out_host["dv"].copy_(dv, non_blocking=True)
+
+        ke = max(3, K // 10)
+        for _ in range(2):
+            e2e_step()
+        barrier(dist, local)
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for _ in range(ke):
+            e2e_step()
+        b.record(stream)
+        torch.cuda.synchronize()
+        barrier(dist, local)
+        e2e_ms = max_over_ranks(dist, a.elapsed_time(b) / ke, dev)
+        h2d = sum(host[n].numel() * host[n].element_size() for n in ("q", "k", "v", "dout"))
+        d2h = sum(t.numel() * t.element_size() for t in out_host.values())
+        e2e = {"value": round(world * f_step / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+               "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+
+    peaks, peak_kind = measured_peaks()
+    bwd_flops = 2.5 * f_fwd
+    achieved = bwd_flops / (bwd_main_ms * 1e-3) / 1e12
+    peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
+    roofline = {"kernel": "bwd_main_kernel<128> (tensor-core backward)", "bound": "tensor",
+                "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
+                "peak_kind": f"bf16 dense, sustained, {peak_kind}", "traffic": recorded_traffic(),
+                "algorithmic_flops_per_launch": bwd_flops, "avg_launch_ms": round(bwd_main_ms, 4)}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        prefix, heads = plan_oracle_sample(15.0)
+        dt, fl = oracle_sample(prefix, heads, args.seed)
+        cpu = {"value": round(fl / dt / 1e12, 6), "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
+               "sample": f"fp64 oracle fwd+bwd on the causal prefix of {prefix} tokens of {heads} heads "
+                         f"(batch element 0, d=128, Q/K std 3), {dt:.1f} s"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded randn; Q/K std 3, V/dO std 1)",
+            "config": {"workload": w.name, "batch": B, "heads": H, "seq_len": N, "head_dim": d, "causal": True,
+                       "global_batch": B * world, "parallelism": f"dp{world} (independent problem per GPU)",
+                       "l2": "no flush: inputs (4 x 134 MB) and outputs exceed the 126 MB L2"},
+            "fwd_tflops": round(world * f_fwd / (fwd_ms * 1e-3) / 1e12, 2),
+            "fwd_ms": round(fwd_ms, 4),
+            "fwd_pct_of_spec_peak": round(100 * f_fwd / (fwd_ms * 1e-3) / 1e12 / SPEC_BF16_TFLOPS, 2),
+            "fwd_bwd_pct_of_spec_peak": round(100 * value / world / SPEC_BF16_TFLOPS, 2),
+            "fwd_bwd_pct_of_measured_peak": round(
+                100 * value / world / float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])), 2),
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches),
+            "gpu_launches_per_step": round(launches / K, 2), "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+# ------------------------------------------------------------ reference arm
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return  # the oracle runs on rank 0's host cores only
+    K, W = args.steps, args.warmup
+    budget = 150.0  # seconds for the whole run
+    prefix, heads = plan_oracle_sample(max(0.05, budget / max(1, K + W)))
+    for _ in range(W):
+        oracle_sample(prefix, heads, args.seed)
+    t = fl = 0.0
+    for _ in range(K):
+        dt, f = oracle_sample(prefix, heads, args.seed)
+        t += dt
+        fl += f
+    value = fl / t / 1e12
+    sample = (f"fp64 oracle fwd+bwd per step on the causal prefix of {prefix} tokens of {heads} heads "
+              f"(batch element 0, d=128, Q/K std 3)")
+    from exact_io_aware_57_b200 import workloads
+
+    w = workloads.WORKLOADS["c3"]
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": K, "warmup": W, "ms_per_step": round(1e3 * t / K, 2), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded randn; Q/K std 3, V/dO std 1)",
+        "config": {"workload": w.name, "batch": w.batch, "heads": w.h_q, "seq_len": w.n, "head_dim": w.d,
+                   "causal": True, "parallelism": "host cores of rank 0"},
+        "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -42,7 +42,11 @@ EXPORTS = {
     "attn_strerror": (ctypes.c_char_p, [_I]),
     "attn_device_status": (_I, [_VP]),
     "attn_launch_count": (_LL, [_I]),
+    "attn_set_kernel_events": (_I, [_I, _VP, _VP]),
 }
+
+ATTN_KERNEL_FWD = 0
+ATTN_KERNEL_BWD = 1
 
 
 class AttnError(RuntimeError):
@@ -186,3 +190,13 @@ def attn_device_status(stream=None) -> int:
 
 def attn_launch_count(reset: bool = False) -> int:
     return int(_lib.attn_launch_count(int(bool(reset))))
+
+
+def attn_set_kernel_events(which: int, start=None, stop=None) -> None:
+    """Record torch.cuda.Event pair (start, stop) around launches of kernel `which`
+    (ATTN_KERNEL_FWD / ATTN_KERNEL_BWD) from this thread; None clears."""
+    sp = None if start is None else start.cuda_event
+    ep = None if stop is None else stop.cuda_event
+    if (start is not None and not sp) or (stop is not None and not ep):
+        raise AttnError("record the events once (torch creates them lazily) before registering them")
+    _check(_lib.attn_set_kernel_events(int(which), sp, ep))

@@ -11,6 +11,7 @@ namespace attn {
 
 namespace {
 thread_local long long g_launches = 0;
+thread_local cudaEvent_t g_kernel_events[2][2] = {{nullptr, nullptr}, {nullptr, nullptr}};
 __device__ int g_status_word;
 
 constexpr int kMaxDevices = 64;
@@ -36,6 +37,11 @@ size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 }  // namespace
 
 void count_launch(int n) { g_launches += n; }
+
+void record_kernel_event(int which, int stop, cudaStream_t st) {
+  cudaEvent_t ev = g_kernel_events[which][stop];
+  if (ev) cudaEventRecord(ev, st);
+}
 
 int* device_status_ptr() {
   int dev = 0;
@@ -318,6 +324,14 @@ int attn_device_status(void* stream) {
   if (cudaMemcpy(&value, ptr, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return ATTN_ERR_CUDA;
   if (cudaMemcpy(ptr, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return ATTN_ERR_CUDA;
   return value;
+}
+
+int attn_set_kernel_events(int which, void* start, void* stop) {
+  if (which != ATTN_KERNEL_FWD && which != ATTN_KERNEL_BWD) return ATTN_ERR_INVALID;
+  if ((start == nullptr) != (stop == nullptr)) return ATTN_ERR_INVALID;
+  g_kernel_events[which][0] = static_cast<cudaEvent_t>(start);
+  g_kernel_events[which][1] = static_cast<cudaEvent_t>(stop);
+  return ATTN_OK;
 }
 
 long long attn_launch_count(int reset) {

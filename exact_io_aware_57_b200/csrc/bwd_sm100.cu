@@ -430,7 +430,9 @@ int launch_main_t(const TcGeom& g, const CUtensorMap& mq, const CUtensorMap& mk,
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return ATTN_ERR_CUDA;
   dim3 grid((g.Nk + BN - 1) / BN, g.Hkv, g.B);
+  record_kernel_event(ATTN_KERNEL_BWD, 0, st);
   kern<<<grid, kThreads, smem, st>>>(mq, mk, mv, mdo, p);
+  record_kernel_event(ATTN_KERNEL_BWD, 1, st);
   count_launch();
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }

@@ -350,7 +350,9 @@ int launch_fwd_t(const TcGeom& g, const CUtensorMap& mq, const CUtensorMap& mk, 
     return ATTN_ERR_CUDA;
   const int max_nq = g.cu_q ? g.max_nq : g.Nq;
   dim3 grid((max_nq + BM - 1) / BM, g.Hq, g.cu_q ? g.num_seqs : g.B);
+  record_kernel_event(ATTN_KERNEL_FWD, 0, st);
   kern<<<grid, kThreads, smem, st>>>(mq, mk, mv, p);
+  record_kernel_event(ATTN_KERNEL_FWD, 1, st);
   count_launch();
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
 }

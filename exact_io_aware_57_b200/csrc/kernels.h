@@ -13,6 +13,9 @@ namespace attn {
 // Launch accounting (per host thread), read by attn_launch_count.
 void count_launch(int n = 1);
 
+// Events recorded around the main forward / backward kernel (measurement hook).
+void record_kernel_event(int which, int stop, cudaStream_t st);
+
 // Default bound on any single in-kernel wait, in SM clock cycles (~1 s).
 constexpr long long kWaitLimitCycles = 2000000000LL;
 

@@ -127,6 +127,18 @@ int attn_device_status(void* stream);
  */
 long long attn_launch_count(int reset);
 
+/*
+ * Measurement hook.  Until cleared, every launch of kernel `which`
+ * (ATTN_KERNEL_FWD: the tensor-core forward kernel; ATTN_KERNEL_BWD: the
+ * tensor-core backward main kernel) issued from the calling host thread is
+ * bracketed by cudaEventRecord(start) / cudaEventRecord(stop) on the launch
+ * stream.  start/stop are caller-owned cudaEvent_t handles; pass NULL for both
+ * to clear.  Returns ATTN_ERR_INVALID for an unknown `which`.
+ */
+#define ATTN_KERNEL_FWD 0
+#define ATTN_KERNEL_BWD 1
+int attn_set_kernel_events(int which, void* start, void* stop);
+
 #ifdef __cplusplus
 }
 #endif
