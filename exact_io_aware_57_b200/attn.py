@@ -35,6 +35,8 @@ EXPORTS = {
     "attn_bwd_workspace_size": (_SZ, [_I, _I, _I, _I]),
     "attn_bwd": (_I, [_VP, _VP, _VP, _FP, _LL, _VP, _FP, _VP, _VP, _VP, _VP, _VP, _SZ, _I, _I, _I, _I, _I,
                       _I, _F, _I, _I, _VP]),
+    "attn_bwd_noalloc": (_I, [_VP, _VP, _VP, _FP, _LL, _VP, _FP, _VP, _VP, _VP, _VP, _I, _I, _I, _I, _I, _I,
+                              _F, _I, _I, _VP]),
     "attn_fwd_varlen": (_I, [_VP, _VP, _VP, _VP, _FP, _IP, _IP, _I, _I, _I, _I, _I, _I, _I, _I, _F, _I, _I,
                              _VP]),
     "attn_naive_scratch_size": (_SZ, [_I, _I]),

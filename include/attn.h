@@ -87,6 +87,29 @@ int attn_bwd(const void* q, const void* k, const void* v, const float* bias,
              void* stream);
 
 /*
+ * attn_bwd without a workspace argument, for callers that cannot allocate
+ * device memory when they run the backward (code inside a framework that owns
+ * all device memory, or latency-critical loops that cannot afford cudaMalloc's
+ * implicit synchronisation).  The pages have no counterpart of this entry
+ * point; it exists for those callers only.
+ *
+ * Arguments, layouts and results are attn_bwd's.  The scratch comes from a
+ * fixed array inside the library (ATTN_NOALLOC_SCRATCH_BYTES per device, held
+ * by every GPU that loads the library until the process exits); nothing is
+ * allocated.  Returns ATTN_ERR_WORKSPACE when attn_bwd_workspace_size(batch,
+ * h_q, n_q, d) exceeds ATTN_NOALLOC_SCRATCH_BYTES.  All calls on a device share
+ * the array: calls that overlap on the GPU race.  The first call on a device
+ * looks up the array's address with that device current; make it before any
+ * stream capture.
+ */
+#define ATTN_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+int attn_bwd_noalloc(const void* q, const void* k, const void* v, const float* bias,
+                     long long bias_batch_stride, const void* o, const float* lse,
+                     const void* dout, void* dq, void* dk, void* dv, int batch, int h_q,
+                     int h_kv, int n_q, int n_k, int d, float scale, int causal, int dtype,
+                     void* stream);
+
+/*
  * Packed variable-length forward.  q: [total_q, h_q, d], k/v: [total_k, h_kv, d],
  * o like q, lse: [h_q, total_q].  cu_seqlens_q / cu_seqlens_k: DEVICE int32
  * arrays of num_seqs + 1 non-decreasing prefix offsets starting at 0; sequence z
