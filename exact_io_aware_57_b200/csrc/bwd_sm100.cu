@@ -1,8 +1,7 @@
-// Backward attention on sm_100a tensor cores: recompute P tile by tile from
-// the stored per-row log-sum-exp ("Attention IO tiling" lesson card, The
-// mechanism: use the retained statistics and permitted recomputation for
-// backward execution; "Understanding FlashAttention Pt 1", 3.6 backward pass:
-// recompute instead of save).  The pages print no gradient formulas; the
+// Backward attention on sm_100a tensor cores: P is rebuilt tile by tile from
+// the per-row log-sum-exp kept by the forward instead of being stored ("Attention
+// IO tiling" lesson card, The mechanism, last step; "Understanding FlashAttention
+// Pt 1", section 3.6 in its contents).  The pages print no gradient formulas; the
 // kernel forms the exact gradient of softmax(scale QK^T + B)V:
 //   P = exp(scale S + B - LSE),  dV = P^T dO,  dP = dO V^T,
 //   dS = P o (dP - D) with D_i = dO_i . O_i,  dQ = scale dS K,  dK = scale dS^T Q.

@@ -2,9 +2,9 @@
 //
 // One CTA owns a tile of 128 query rows of one (batch or sequence, head) and
 // streams 128-key tiles of K and V past it ("Attention IO tiling" lesson card,
-// The mechanism: partition into tiles that fit the local-memory budget, form
-// one score block, update running softmax statistics, accumulate weighted
-// values while rescaling, discard the score block).
+// The mechanism: Q/K/V are cut into on-chip-sized tiles; each score tile
+// updates the per-row softmax state and the rescaled value sum, then is
+// dropped rather than stored).
 //
 //   warp 0      TMA producer: Q once, then K_j / V_j into a 2-stage smem ring
 //   warp 1      TMEM owner + single-thread tcgen05.mma issuer
@@ -21,7 +21,8 @@
 // Normalizer", in base 2), writes P to TMEM and -- once the previous P V has
 // landed -- rescales the O accumulator by 2^(m - m') when the max moved.  The
 // MMA warp then accumulates O += P V_j.  O / l and LSE = (m + log2 l) ln 2 are
-// written once at the end ("normalize once at the end", the same page's lab).
+// written once, after the last tile (the division by l happens a single time,
+// as in the same page's lab).
 // Causal: KV tiles that lie wholly above the diagonal are never loaded.
 #include <algorithm>
 

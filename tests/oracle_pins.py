@@ -5,8 +5,8 @@ real oracle (test_oracle_pins.py) and on variants with planted mistakes
 
 Sources:
   * merge recurrence == one-shot softmax: "Softmax does not need the matrix",
-    "Carry the Normalizer" (the (m, l, a) state is enough to continue the exact
-    softmax later) and its lab (materialised vs online-tiled row agree);
+    "Carry the Normalizer" (the carried (m, l, a) state suffices to resume the
+    softmax without error) and its lab (materialised and streamed rows agree);
   * constant scores / single key / causal row 0 / permutation and shift
     invariance: closed forms of the softmax definition (same page and the
     handbook's 0.2 Notation);
