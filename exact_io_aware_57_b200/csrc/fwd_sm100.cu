@@ -39,6 +39,7 @@ constexpr int NST = 2;           // K/V smem stages
 constexpr int kThreads = 192;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColO = 256, kColP = 384;
+constexpr float kRescaleThreshold = 8.f;  // log2 units: P stays <= 256
 
 template <int D>
 struct FwdSmem {
@@ -48,7 +49,7 @@ struct FwdSmem {
   alignas(1024) uint8_t v[NST][kTileBytes];
   uint64_t q_full;
   uint64_t k_full[NST], k_empty[NST], v_full[NST], v_empty[NST];
-  uint64_t s_full[2], s_free[2], p_full[2];
+  uint64_t s_full[2], p_full[2];
   uint64_t pv_done, drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -76,7 +77,7 @@ ATTN_DEVINL void reg_fence(uint32_t (&r)[N]) {
   for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
 }
 
-template <int D, bool HAS_BIAS>
+template <int D, bool HAS_BIAS, bool FAST>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -118,7 +119,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&s.s_full[i], 1);
-      mbar_init(&s.s_free[i], 4);
       mbar_init(&s.p_full[i], 4);
     }
     mbar_init(&s.pv_done, 1);
@@ -176,7 +176,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t q_addr = smem_u32(s.q);
       auto issue_s = [&](int j) -> bool {
         const int buf = j & 1, st = j % NST;
-        if (j >= 2 && !mbar_wait(&s.s_free[buf], ((j >> 1) - 1) & 1, ab)) return false;
         if (!mbar_wait(&s.k_full[st], (j / NST) & 1, ab)) return false;
         tc_fence_after();
         const uint32_t k_addr = smem_u32(s.k[st]);
@@ -195,17 +194,33 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (ok && n_kv > 1) ok = issue_s(1);
       for (int j = 0; ok && j < n_kv; ++j) {
         const int buf = j & 1, st = j % NST;
+        // p_full(j): P_j is in TMEM, O is rescaled, and S buffer `buf` has been read
         if (!mbar_wait(&s.p_full[buf], (j >> 1) & 1, ab)) break;
         if (!mbar_wait(&s.v_full[st], (j / NST) & 1, ab)) break;
+        const bool next = j + 2 < n_kv;
+        const int st2 = (j + 2) % NST;
+        if (next && !mbar_wait(&s.k_full[st2], ((j + 2) / NST) & 1, ab)) break;
         tc_fence_after();
-        const uint32_t v_addr = smem_u32(s.v[st]);
+        const uint32_t v_addr = smem_u32(s.v[st]), k_addr = smem_u32(s.k[st2]);
+        // O += P_j V_j interleaved with S_{j+2} = Q K_{j+2}^T: two independent
+        // accumulators keep the tensor pipe busy (a chain of MMAs into one
+        // accumulator waits on each previous result)
 #pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk)
+        for (int kk = 0; kk < BN / 16; ++kk) {
           mma_ts(tmem + kColO, tmem + kColP + buf * 64 + kk * 8, sdesc_sw128(v_addr + kk * 2048, BN * 128, 1024),
                  idesc_pv, (j > 0 || kk > 0));
+          if (next && kk < D / 16) {
+            const uint32_t off = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
+            mma_ss(tmem + kColS + buf * BN, sdesc_sw128(q_addr + off, 16, 1024),
+                   sdesc_sw128(k_addr + off, 16, 1024), idesc_s, kk > 0);
+          }
+        }
         mma_commit(&s.pv_done);
         mma_commit(&s.v_empty[st]);
-        if (j + 2 < n_kv && !issue_s(j + 2)) break;
+        if (next) {
+          mma_commit(&s.s_full[buf]);
+          mma_commit(&s.k_empty[st2]);
+        }
       }
       // TMEM must be quiescent before it is released
       mma_commit(&s.drain);
@@ -222,6 +237,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     if constexpr (HAS_BIAS) {
       if (row_ok) brow = p.bias + bidx * p.bias_bstride + ((long long)h * p.Nq + i) * p.Nk;
     }
+    // m: the reference max of the row (log2 units) that P and l are expressed
+    // against.  It only moves when a tile's max exceeds it by more than
+    // kRescaleThreshold, so P <= 2^threshold and O is rescaled rarely; the
+    // final O / l and LSE do not depend on which reference was used.
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int j = 0; j < n_kv; ++j) {
@@ -229,56 +248,68 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(&s.s_full[buf], (j >> 1) & 1, ab));
       if (!ok) break;
       tc_fence_after();
-      uint32_t sr[4][32];
+      uint32_t sr[BN];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_off + kColS + buf * BN + c * 32, sr[c]);
+      for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_off + kColS + buf * BN + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
       tmem_wait_ld();
-#pragma unroll
-      for (int c = 0; c < 4; ++c) reg_fence(sr[c]);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s.s_free[buf]);
-
-      // scale (+ bias) in log2 units, mask, row max of the block
+      reg_fence(sr);
       const int kbase = j * BN;
-      const bool need_mask = (kbase + BN > len_k) || (p.causal && kbase + BN - 1 > m0 + diag);
-      float t[BN];
-      float mb = -INFINITY;
+      if constexpr (!FAST) {
+        // general scores: t = s * scale * log2(e) (+ bias * log2(e))
 #pragma unroll
-      for (int c = 0; c < BN; ++c) {
-        float x = __uint_as_float(sr[c >> 5][c & 31]) * p.scale_log2;
-        if constexpr (HAS_BIAS) {
-          if (brow != nullptr && kbase + c < len_k) x = fmaf(__ldg(brow + kbase + c), kLog2e, x);
+        for (int c = 0; c < BN; ++c) {
+          float x = __uint_as_float(sr[c]) * p.scale_log2;
+          if constexpr (HAS_BIAS) {
+            if (brow != nullptr && kbase + c < len_k) x = fmaf(__ldg(brow + kbase + c), kLog2e, x);
+          }
+          sr[c] = __float_as_uint(x);
         }
-        if (need_mask) {
-          const int key = kbase + c;
-          if (key >= len_k || (p.causal && key > i + diag)) x = -INFINITY;
-        }
-        t[c] = x;
-        mb = fmaxf(mb, x);
       }
-      const float m_new = fmaxf(m, mb);
-      const float m_use = m_new == -INFINITY ? 0.f : m_new;
-      const float alpha = ex2(m - m_use);
-      float rowsum = 0.f;
-      uint32_t pk[2][32];
+      if ((kbase + BN > len_k) || (p.causal && kbase + BN - 1 > m0 + diag)) {
+        // diagonal or ragged tile: hide invisible keys
+        const int lim = min(len_k, p.causal ? i + diag + 1 : len_k) - kbase;
+#pragma unroll
+        for (int c = 0; c < BN; ++c)
+          if (c >= lim) sr[c] = 0xff800000u;  // -inf
+      }
+      float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < BN; c += 2) {
+        mx0 = fmaxf(mx0, __uint_as_float(sr[c]));
+        mx1 = fmaxf(mx1, __uint_as_float(sr[c + 1]));
+      }
+      float mx = fmaxf(mx0, mx1);
+      if constexpr (FAST) mx *= p.scale_log2;  // scale > 0: max commutes with it
+      const bool move = mx > m + kRescaleThreshold;
+      const float m_next = move ? mx : m;
+      const float alpha = move ? ex2(m - m_next) : 1.f;
+      const float neg_m = m_next == -INFINITY ? 0.f : -m_next;
+      float rs0 = 0.f, rs1 = 0.f;
+      uint32_t pk[BN / 2];
 #pragma unroll
       for (int c = 0; c < BN / 2; ++c) {
-        const float p0 = ex2(t[2 * c] - m_use), p1 = ex2(t[2 * c + 1] - m_use);
-        rowsum += p0 + p1;
-        pk[c >> 5][c & 31] = pack_bf16(p0, p1);
+        float p0, p1;
+        if constexpr (FAST) {
+          p0 = ex2(fmaf(__uint_as_float(sr[2 * c]), p.scale_log2, neg_m));
+          p1 = ex2(fmaf(__uint_as_float(sr[2 * c + 1]), p.scale_log2, neg_m));
+        } else {
+          p0 = ex2(__uint_as_float(sr[2 * c]) + neg_m);
+          p1 = ex2(__uint_as_float(sr[2 * c + 1]) + neg_m);
+        }
+        rs0 += p0;
+        rs1 += p1;
+        pk[c] = pack_bf16(p0, p1);
       }
-      l = l * alpha + rowsum;
-      // P buffer `buf` was last read by P V_{j-2}, which completed before the
-      // previous iteration's pv_done wait returned.
-      tmem_st32(tmem + lane_off + kColP + buf * 64, pk[0]);
-      tmem_st32(tmem + lane_off + kColP + buf * 64 + 32, pk[1]);
+      l = l * alpha + (rs0 + rs1);
+      m = m_next;
       if (j > 0) {
+        // P V_{j-1} must be done before O is rescaled and before the P buffer
+        // it read two steps ago is reused.
         ok = __all_sync(0xffffffffu, mbar_wait(&s.pv_done, (j - 1) & 1, ab));
         if (!ok) break;
         tc_fence_after();
         if (__any_sync(0xffffffffu, alpha != 1.f)) {
-#pragma unroll
+#pragma unroll 1
           for (int c = 0; c < D / 32; ++c) {
             uint32_t orr[32];
             tmem_ld32(tmem + lane_off + kColO + c * 32, orr);
@@ -290,7 +321,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      m = m_new;
+      tmem_st32(tmem + lane_off + kColP + buf * 64, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+      tmem_st32(tmem + lane_off + kColP + buf * 64 + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -340,13 +372,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D, bool HAS_BIAS>
+template <int D, bool HAS_BIAS, bool FAST>
 int launch_fwd_t(const TcGeom& g, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                  const FwdParams& p, cudaStream_t st) {
   // At least half of the SM's shared memory, so that a second CTA never waits
   // on the 512 TMEM columns this one holds.
   const size_t smem = std::max<size_t>(sizeof(FwdSmem<D>) + 1024, 116 * 1024);
-  auto kern = fwd_sm100_kernel<D, HAS_BIAS>;
+  auto kern = fwd_sm100_kernel<D, HAS_BIAS, FAST>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return ATTN_ERR_CUDA;
   const int max_nq = g.cu_q ? g.max_nq : g.Nq;
@@ -395,10 +427,14 @@ int launch_fwd_sm100(const TcGeom& g, __nv_bfloat16* o, float* lse, cudaStream_t
   p.status = device_status_ptr();
   p.wait_limit = kWaitLimitCycles;
   if (!p.status) return ATTN_ERR_CUDA;
-  const bool has_bias = g.bias != nullptr;
-  if (g.D == 64)
-    return has_bias ? launch_fwd_t<64, true>(g, mq, mk, mv, p, st) : launch_fwd_t<64, false>(g, mq, mk, mv, p, st);
-  return has_bias ? launch_fwd_t<128, true>(g, mq, mk, mv, p, st) : launch_fwd_t<128, false>(g, mq, mk, mv, p, st);
+  // FAST: no bias and a positive scale, so the row max can be taken on raw scores
+  const bool has_bias = g.bias != nullptr, fast = !has_bias && g.scale > 0.f;
+  if (g.D == 64) {
+    if (has_bias) return launch_fwd_t<64, true, false>(g, mq, mk, mv, p, st);
+    return fast ? launch_fwd_t<64, false, true>(g, mq, mk, mv, p, st) : launch_fwd_t<64, false, false>(g, mq, mk, mv, p, st);
+  }
+  if (has_bias) return launch_fwd_t<128, true, false>(g, mq, mk, mv, p, st);
+  return fast ? launch_fwd_t<128, false, true>(g, mq, mk, mv, p, st) : launch_fwd_t<128, false, false>(g, mq, mk, mv, p, st);
 }
 
 }  // namespace attn
