@@ -17,7 +17,7 @@
 //   warp 0      TMA producer (K_j, V_j once; Q_i, dO_i per step) + LSE/D rows
 //   warp 1      TMEM owner + single-thread tcgen05.mma issuer
 //   warps 2..5  thread t owns key row t: P^T, dS^T, and the dK/dV epilogue
-//   warps 6..9  thread t owns query row t of the dQ tile: TMEM -> fp32 reductions
+//   warps 6..9  thread t owns query row t of the dQ tile: TMEM -> smem -> TMA reduce-add
 // TMEM columns: [0,128) S^T (then P^T as bf16 pairs in [0,64)),
 //   [128,256) dP^T (then the dQ tile), [256,256+D) dV, [256+D,256+2D) dK.
 // Per step (query head h, query tile i):
@@ -25,7 +25,7 @@
 //   WG0   P^T = 2^(scale log2e S^T + log2e B^T - log2e LSE) -> TMEM (bf16);
 //         dS^T = P^T o (dP^T - D) -> shared memory (bf16, 128B-swizzled)
 //   MMA   dV += P^T dO_i (P^T from TMEM), dK += dS^T Q_i, dQ_i = dS K_j
-//   WG1   dQ_i -> red.global.add into the fp32 accumulator
+//   WG1   dQ_i -> shared memory -> TMA bulk reduce-add into the fp32 accumulator
 #include <algorithm>
 
 #include "common.cuh"
@@ -50,8 +50,8 @@ struct BwdSmem {
   alignas(1024) uint8_t q[NSTQ][kTileBytes];
   alignas(1024) uint8_t dout[NSTQ][kTileBytes];
   alignas(1024) uint8_t ds[128 * 128 * 2];  // dS^T, [key][query] in two 64-column blocks
-  float lse2[NSTQ][BM];                     // log2(e) * LSE of the step's query rows (+inf: no key)
-  float drow[NSTQ][BM];                     // D_i of the step's query rows
+  alignas(16) float nlse2[NSTQ][BM];        // -log2(e) * LSE of the step's query rows (-inf: no key)
+  alignas(16) float drow[NSTQ][BM];         // D_i of the step's query rows
   uint64_t kv_full, q_full[NSTQ], q_empty[NSTQ];
   uint64_t s_full, ds_ready, dq_full, dq_drained, drain;
   uint32_t tmem_base;
@@ -79,20 +79,90 @@ ATTN_DEVINL void reg_fence(uint32_t (&r)[N]) {
   for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
 }
 
-ATTN_DEVINL void red_add_v4(float* addr, float a, float b, float c, float d) {
-  asm volatile("red.relaxed.gpu.global.add.v4.f32 [%0], {%1,%2,%3,%4};" ::"l"(addr), "f"(a), "f"(b), "f"(c), "f"(d)
-               : "memory");
+
+// out[tile] += smem tile (fp32), completion tracked by bulk groups
+ATTN_DEVINL void tma_reduce_add_4d(const CUtensorMap* map, const void* src, int c0, int c1, int c2, int c3) {
+  asm volatile(
+      "cp.reduce.async.bulk.tensor.4d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(smem_u32(src)), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+      : "memory");
 }
+ATTN_DEVINL void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+ATTN_DEVINL void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+ATTN_DEVINL void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+// non-.aligned form: legal even if the calling warp arrives diverged
+ATTN_DEVINL void named_bar_sync(int id, int n) { asm volatile("barrier.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
 
 ATTN_DEVINL void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+
+// P^T and dS^T for one key row (this thread) and 128 queries, 32 at a time:
+//   P^T = 2^(scale log2e s + log2e B - log2e LSE), dS^T = P^T (dP^T - D);
+// P^T goes back into TMEM (bf16 pairs, A operand of dV += P^T dO) and dS^T
+// into the 128B-swizzled shared tile.  MASK zeroes queries this key is hidden
+// from (causal: query i sees key j iff j <= i + diag; padding rows and keys).
+template <bool MASK, bool HAS_BIAS>
+ATTN_DEVINL void bwd_chunks(uint32_t st_col, uint32_t dp_col, const float* nlse2, const float* drow, uint32_t ds_row,
+                            int r, float scale_log2, const float* bcol, int nk, int i0, int len_q, int kj, int len_k,
+                            int diag) {
+#pragma unroll 1
+  for (int c = 0; c < BM / 32; ++c) {
+    uint32_t sr[32], dpr[32];
+    tmem_ld32(st_col + c * 32, sr);
+    tmem_ld32(dp_col + c * 32, dpr);
+    tmem_wait_ld();
+    reg_fence(sr);
+    reg_fence(dpr);
+    const float4* nl4 = reinterpret_cast<const float4*>(nlse2 + c * 32);
+    const float4* dr4 = reinterpret_cast<const float4*>(drow + c * 32);
+    // queries q0 + e with e < vis are visible from this key
+    const int q0 = i0 + c * 32;
+    int vis_lo = 0, vis_hi = 32;
+    if constexpr (MASK) {
+      vis_lo = kj - diag - q0;                 // causal: q >= kj - diag
+      vis_hi = min(32, len_q - q0);            // padding queries
+      if (kj >= len_k) vis_hi = 0;             // padding key
+    }
+    uint32_t pk[16], dk[16];
+#pragma unroll
+    for (int e4 = 0; e4 < 8; ++e4) {
+      const float4 nl = nl4[e4], dr = dr4[e4];
+      const float nlv[4] = {nl.x, nl.y, nl.z, nl.w}, drv[4] = {dr.x, dr.y, dr.z, dr.w};
+      float pv[4], dsv[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int e = e4 * 4 + u;
+        float t = fmaf(__uint_as_float(sr[e]), scale_log2, nlv[u]);
+        if constexpr (HAS_BIAS) t = fmaf(__ldg(bcol + (long long)min(q0 + e, len_q - 1) * nk), kLog2e, t);
+        float pe = ex2(t);
+        if constexpr (MASK) pe = (e >= vis_lo && e < vis_hi) ? pe : 0.f;
+        pv[u] = pe;
+        dsv[u] = pe * (__uint_as_float(dpr[e]) - drv[u]);
+      }
+      pk[2 * e4] = pack_bf16(pv[0], pv[1]);
+      pk[2 * e4 + 1] = pack_bf16(pv[2], pv[3]);
+      dk[2 * e4] = pack_bf16(dsv[0], dsv[1]);
+      dk[2 * e4 + 1] = pack_bf16(dsv[2], dsv[3]);
+    }
+    // P^T columns [16c, 16c+16) lie in S^T columns already read
+    tmem_st16(st_col + c * 16, pk);
+    // dS^T: 32 queries = 4 chunks of 16 bytes in 64-column block c/2
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int chunk = (c & 1) * 4 + u;  // 16-byte chunk within the 128-byte row
+      const uint32_t addr = ds_row + (c >> 1) * (128 * 128) + ((chunk ^ (r & 7)) << 4);
+      st_shared_v4(addr, dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
+    }
+  }
 }
 
 template <int D, bool HAS_BIAS>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
-                    const BwdParams p) {
+                    const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
   using Smem = BwdSmem<D>;
   constexpr int KB = D / 64;
   constexpr uint32_t kColDK = kColDV + D;
@@ -176,13 +246,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int e = 0; e < BM / 32; ++e) {
         const int c = lane + 32 * e;
         const int qi = i0 + c;
-        float l2 = INFINITY, dr = 0.f;
+        float l2 = -INFINITY, dr = 0.f;
         if (qi < len_q) {
           const float lse = p.lse[row0 + qi];
-          l2 = lse == -INFINITY ? INFINITY : lse * kLog2e;
+          l2 = lse == -INFINITY ? -INFINITY : -lse * kLog2e;
           dr = p.drow[row0 + qi];
         }
-        s.lse2[st][c] = l2;
+        s.nlse2[st][c] = l2;
         s.drow[st][c] = dr;
       }
       mbar_arrive(&s.q_full[st]);
@@ -204,43 +274,36 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int step = 0; ok && step < n_steps; ++step) {
         const int st = step % NSTQ;
         if (!mbar_wait(&s.q_full[st], (step / NSTQ) & 1, ab)) break;
-        // dQ of the previous step must have left TMEM (it lives where dP^T goes)
+        // dQ of the previous step must have left TMEM (it lives where dP^T goes);
+        // its commit also covers every earlier MMA, so P^T in S^T's columns is free
         if (step > 0 && !mbar_wait(&s.dq_drained, (step - 1) & 1, ab)) break;
         tc_fence_after();
         const uint32_t q_addr = smem_u32(s.q[st]), do_addr = smem_u32(s.dout[st]);
+        // S^T = K_j Q_i^T and dP^T = V_j dO_i^T, interleaved (independent accumulators)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
           mma_ss(tmem + kColST, sdesc_sw128(k_addr + off, 16, 1024), sdesc_sw128(q_addr + off, 16, 1024), idesc_s,
                  kk > 0);
-        }
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
           mma_ss(tmem + kColDPT, sdesc_sw128(v_addr + off, 16, 1024), sdesc_sw128(do_addr + off, 16, 1024),
                  idesc_s, kk > 0);
         }
         mma_commit(&s.s_full);
         if (!mbar_wait(&s.ds_ready, step & 1, ab)) break;
         tc_fence_after();
-        // dV += P^T dO_i   (A: P^T bf16 in TMEM, K = query)
-#pragma unroll
-        for (int kk = 0; kk < BM / 16; ++kk)
-          mma_ts(tmem + kColDV, tmem + kColST + kk * 8, sdesc_sw128(do_addr + kk * 2048, BM * 128, 1024), idesc_kv,
-                 (step > 0 || kk > 0));
-        // dK += dS^T Q_i  (A: dS^T in shared memory, K-major over queries)
+        // dV += P^T dO_i (P^T from TMEM), dK += dS^T Q_i, dQ_i = dS K_j (dS^T read
+        // MN-major): three accumulators, issued round-robin
 #pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk) {
           const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+          mma_ts(tmem + kColDV, tmem + kColST + kk * 8, sdesc_sw128(do_addr + kk * 2048, BM * 128, 1024), idesc_kv,
+                 (step > 0 || kk > 0));
           mma_ss(tmem + kColDK, sdesc_sw128(ds_addr + off, 16, 1024), sdesc_sw128(q_addr + kk * 2048, BM * 128, 1024),
                  idesc_kv, (step > 0 || kk > 0));
-        }
-        mma_commit(&s.q_empty[st]);
-        // dQ_i = dS K_j  (A: the same dS^T buffer read MN-major, K = key)
-#pragma unroll
-        for (int kk = 0; kk < BN / 16; ++kk)
           mma_ss(tmem + kColDPT, sdesc_sw128(ds_addr + kk * 2048, 128 * 128, 1024),
                  sdesc_sw128(k_addr + kk * 2048, BN * 128, 1024), idesc_dq, kk > 0);
+        }
+        mma_commit(&s.q_empty[st]);
         mma_commit(&s.dq_full);
       }
       mma_commit(&s.drain);
@@ -262,49 +325,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!ok) break;
       // q_full for this stage completed before s_full (the MMA waited on it)
       tc_fence_after();
-      const bool need_mask = (kj >= len_k) || (i0 + BM > len_q) || (p.causal && n0 + BN - 1 > i0 + diag);
+      // tile-level (warp-uniform) condition: the two chunk variants hold
+      // warp-collective tcgen05 instructions, so every lane must take the same one
+      const bool need_mask = (n0 + BN > len_k) || (i0 + BM > len_q) || (p.causal && n0 + BN - 1 > i0 + diag);
       const float* bcol = nullptr;
-      if constexpr (HAS_BIAS) {
-        if (kj < len_k) bcol = p.bias + b * p.bias_bstride + (long long)h * p.Nq * p.Nk + kj;
-      }
-#pragma unroll
-      for (int c = 0; c < BM / 32; ++c) {
-        uint32_t sr[32], dpr[32];
-        tmem_ld32(tmem + lane_off + kColST + c * 32, sr);
-        tmem_ld32(tmem + lane_off + kColDPT + c * 32, dpr);
-        tmem_wait_ld();
-        reg_fence(sr);
-        reg_fence(dpr);
-        uint32_t pk[16], dk[16];
-#pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          float pv[2], dsv[2];
-#pragma unroll
-          for (int u = 0; u < 2; ++u) {
-            const int col = c * 32 + e + u;
-            const int qi = i0 + col;
-            float t = __uint_as_float(sr[e + u]) * p.scale_log2 - s.lse2[st][col];
-            if constexpr (HAS_BIAS) {
-              if (bcol != nullptr && qi < len_q) t = fmaf(__ldg(bcol + (long long)qi * p.Nk), kLog2e, t);
-            }
-            float pe = ex2(t);
-            if (need_mask && (kj >= len_k || qi >= len_q || (p.causal && kj > qi + diag))) pe = 0.f;
-            pv[u] = pe;
-            dsv[u] = pe * (__uint_as_float(dpr[e + u]) - s.drow[st][col]);
-          }
-          pk[e >> 1] = pack_bf16(pv[0], pv[1]);
-          dk[e >> 1] = pack_bf16(dsv[0], dsv[1]);
-        }
-        // P^T columns [16c, 16c+16) lie in S^T columns already read
-        tmem_st16(tmem + lane_off + kColST + c * 16, pk);
-        // dS^T: 32 queries = 4 chunks of 16 bytes in 64-column block c/2
-#pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int chunk = (c & 1) * 4 + u;  // 16-byte chunk within the 128-byte row
-          const uint32_t addr = ds_row + (c >> 1) * (128 * 128) + ((chunk ^ (r & 7)) << 4);
-          st_shared_v4(addr, dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
-        }
-      }
+      if constexpr (HAS_BIAS) bcol = p.bias + b * p.bias_bstride + (long long)h * p.Nq * p.Nk + min(kj, len_k - 1);
+      // 32 queries per pass; a rolled loop keeps the code small enough for the
+      // instruction cache, and the masked variant is chosen once per step so the
+      // element loop has no branches
+      const uint32_t st_col = tmem + lane_off + kColST, dp_col = tmem + lane_off + kColDPT;
+      if (need_mask)
+        bwd_chunks<true, HAS_BIAS>(st_col, dp_col, s.nlse2[st], s.drow[st], ds_row, r, p.scale_log2, bcol, p.Nk, i0,
+                                   len_q, kj, len_k, p.causal ? diag : (1 << 30));
+      else
+        bwd_chunks<false, HAS_BIAS>(st_col, dp_col, s.nlse2[st], s.drow[st], ds_row, r, p.scale_log2, bcol, p.Nk, i0,
+                                    len_q, kj, len_k, 1 << 30);
       tmem_wait_st();
       fence_proxy_async_smem();
       tc_fence_before();
@@ -346,32 +381,54 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ===================================================== dQ drain (thread = query row)
+    // dQ_i leaves TMEM through the (now idle) dS^T shared tile, 64 columns per
+    // pass, and is added to the fp32 accumulator by TMA bulk reductions.
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
+    const bool leader = warp == 6 && lane == 0;
+    const uint32_t stage_row = smem_u32(s.ds) + r * 128;
     for (int step = 0; step < n_steps; ++step) {
       const int h = hk * G + step / per_head;
-      const int qi = (i_first + step % per_head) * BM + r;
+      const int i0 = (i_first + step % per_head) * BM;
       if (!__all_sync(0xffffffffu, mbar_wait(&s.dq_full, step & 1, ab))) break;
       tc_fence_after();
-      float* dst = p.dq_acc + (((long long)b * p.Nq + qi) * p.Hq + h) * D;
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        uint32_t a[32];
-        tmem_ld32(tmem + lane_off + kColDPT + c * 32, a);
-        tmem_wait_ld();
-        reg_fence(a);
-        if (qi < len_q) {
-#pragma unroll
-          for (int e = 0; e < 32; e += 4)
-            red_add_v4(dst + c * 32 + e, __uint_as_float(a[e]), __uint_as_float(a[e + 1]), __uint_as_float(a[e + 2]),
-                       __uint_as_float(a[e + 3]));
+#pragma unroll 1
+      for (int pass = 0; pass < D / 64; ++pass) {
+        if (pass > 0) {
+          if (leader) bulk_wait_read0();  // the previous pass's reductions have read the tile
+          __syncwarp();
+          named_bar_sync(1, 128);
         }
+#pragma unroll
+        for (int cc = 0; cc < 2; ++cc) {
+          uint32_t a[32];
+          tmem_ld32(tmem + lane_off + kColDPT + (pass * 2 + cc) * 32, a);
+          tmem_wait_ld();
+          reg_fence(a);
+          // 32 fp32 = 8 chunks of 16 bytes, 128B-swizzled like the TMA box
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            st_shared_v4(stage_row + cc * (128 * 128) + ((u ^ (r & 7)) << 4), a[4 * u], a[4 * u + 1], a[4 * u + 2],
+                         a[4 * u + 3]);
+        }
+        fence_proxy_async_smem();
+        named_bar_sync(1, 128);
+        if (leader) {
+#pragma unroll
+          for (int cc = 0; cc < 2; ++cc)
+            tma_reduce_add_4d(&tm_dq, s.ds + cc * (128 * 128), (pass * 2 + cc) * 32, h, i0, b);
+          bulk_commit();
+        }
+        __syncwarp();
       }
-      tc_fence_before();
+      // the next step's dS^T overwrites the staging tile: wait until it was read
+      if (leader) bulk_wait_read0();
       __syncwarp();
+      tc_fence_before();
       if (lane == 0) mbar_arrive(&s.dq_drained);
     }
+    if (leader) bulk_wait0();
   }
 
   tc_fence_before();
@@ -423,14 +480,14 @@ __global__ void __launch_bounds__(256) bwd_dq_kernel(const float* __restrict__ a
 
 template <int D, bool HAS_BIAS>
 int launch_main_t(const TcGeom& g, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                  const CUtensorMap& mdo, const BwdParams& p, cudaStream_t st) {
+                  const CUtensorMap& mdo, const CUtensorMap& mdq, const BwdParams& p, cudaStream_t st) {
   const size_t smem = std::max<size_t>(sizeof(BwdSmem<D>), 116 * 1024);
   auto kern = bwd_main_kernel<D, HAS_BIAS>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return ATTN_ERR_CUDA;
   dim3 grid((g.Nk + BN - 1) / BN, g.Hkv, g.B);
   record_kernel_event(ATTN_KERNEL_BWD, 0, st);
-  kern<<<grid, kThreads, smem, st>>>(mq, mk, mv, mdo, p);
+  kern<<<grid, kThreads, smem, st>>>(mq, mk, mv, mdo, mdq, p);
   record_kernel_event(ATTN_KERNEL_BWD, 1, st);
   count_launch();
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
@@ -454,13 +511,18 @@ int launch_bwd_sm100(const TcGeom& g, const __nv_bfloat16* o, const float* lse, 
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   }
   // 2) main
-  CUtensorMap mq, mk, mv, mdo;
+  CUtensorMap mq, mk, mv, mdo, mdq;
   const uint32_t box[4] = {64, 1, 128, 1};
   {
     const uint64_t dims[4] = {(uint64_t)g.D, (uint64_t)g.Hq, (uint64_t)g.Nq, (uint64_t)g.B};
     const uint64_t str[3] = {(uint64_t)g.D * 2, (uint64_t)g.Hq * g.D * 2, (uint64_t)g.Nq * g.Hq * g.D * 2};
     if (encode_tmap_bf16(&mq, g.q, 4, dims, str, box) != ATTN_OK) return ATTN_ERR_CUDA;
     if (encode_tmap_bf16(&mdo, dout, 4, dims, str, box) != ATTN_OK) return ATTN_ERR_CUDA;
+    // fp32 accumulator: 32 floats (128 bytes) x 128 rows per box
+    const uint64_t str32[3] = {(uint64_t)g.D * 4, (uint64_t)g.Hq * g.D * 4, (uint64_t)g.Nq * g.Hq * g.D * 4};
+    const uint32_t box32[4] = {32, 1, 128, 1};
+    if (encode_tmap(&mdq, dq_acc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dims, str32, box32) != ATTN_OK)
+      return ATTN_ERR_CUDA;
   }
   {
     const uint64_t dims[4] = {(uint64_t)g.D, (uint64_t)g.Hkv, (uint64_t)g.Nk, (uint64_t)g.B};
@@ -489,10 +551,10 @@ int launch_bwd_sm100(const TcGeom& g, const __nv_bfloat16* o, const float* lse, 
   int rc;
   const bool hb = g.bias != nullptr;
   if (g.D == 64)
-    rc = hb ? launch_main_t<64, true>(g, mq, mk, mv, mdo, p, st) : launch_main_t<64, false>(g, mq, mk, mv, mdo, p, st);
+    rc = hb ? launch_main_t<64, true>(g, mq, mk, mv, mdo, mdq, p, st) : launch_main_t<64, false>(g, mq, mk, mv, mdo, mdq, p, st);
   else
-    rc = hb ? launch_main_t<128, true>(g, mq, mk, mv, mdo, p, st)
-            : launch_main_t<128, false>(g, mq, mk, mv, mdo, p, st);
+    rc = hb ? launch_main_t<128, true>(g, mq, mk, mv, mdo, mdq, p, st)
+            : launch_main_t<128, false>(g, mq, mk, mv, mdo, mdq, p, st);
   if (rc) return rc;
   // 3) dQ
   const long long n8 = (long long)g.B * g.Nq * g.Hq * g.D / 8;

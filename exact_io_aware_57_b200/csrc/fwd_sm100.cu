@@ -233,10 +233,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int i = m0 + r;                 // row inside its sequence
     const bool row_ok = i < len_q;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const float* brow = nullptr;
-    if constexpr (HAS_BIAS) {
-      if (row_ok) brow = p.bias + bidx * p.bias_bstride + ((long long)h * p.Nq + i) * p.Nk;
-    }
+    const float* brow = nullptr;  // rows past the end read the last row (their output is dropped)
+    if constexpr (HAS_BIAS) brow = p.bias + bidx * p.bias_bstride + ((long long)h * p.Nq + min(i, len_q - 1)) * p.Nk;
     // m: the reference max of the row (log2 units) that P and l are expressed
     // against.  It only moves when a tile's max exceeds it by more than
     // kRescaleThreshold, so P <= 2^threshold and O is rescaled rarely; the
@@ -259,9 +257,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < BN; ++c) {
           float x = __uint_as_float(sr[c]) * p.scale_log2;
-          if constexpr (HAS_BIAS) {
-            if (brow != nullptr && kbase + c < len_k) x = fmaf(__ldg(brow + kbase + c), kLog2e, x);
-          }
+          if constexpr (HAS_BIAS) x = fmaf(__ldg(brow + min(kbase + c, len_k - 1)), kLog2e, x);
           sr[c] = __float_as_uint(x);
         }
       }

@@ -63,5 +63,7 @@ int launch_fwd_naive(const TcGeom& g, __nv_bfloat16* o, float* lse, float* s_scr
 // Tensor-map encoding (driver entry point resolved at run time).
 int encode_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
                      const uint64_t* strides_bytes, const uint32_t* box);
+int encode_tmap(CUtensorMap* map, const void* base, CUtensorMapDataType dtype, int rank, const uint64_t* dims,
+                const uint64_t* strides_bytes, const uint32_t* box);
 
 }  // namespace attn

@@ -85,3 +85,16 @@ def test_fwd_full_size_mha_d64(orc):
     eo, el = check_fwd_sampled(orc, inp.q, inp.k, inp.v, o.cpu(), lse.cpu(), False,
                                [(0, 0), (1, 7), (3, 15)], sample_rows(2048))
     assert eo <= TOL_O_BF16 and el <= TOL_LSE_BF16, (eo, el)
+
+
+@pytest.mark.parametrize("d,causal", [(128, True), (64, False)])
+def test_fwd_naive_comparator(orc, d, causal):
+    """The materialising three-kernel comparator computes the same function."""
+    from exact_io_aware_57_b200 import attn
+
+    inp = synth.make_dense(2, 4, 2, 300, 300, d, with_dout=False, seed=9)
+    o, lse = attn.attn_fwd_naive(inp.q.cuda(), inp.k.cuda(), inp.v.cuda(), causal=causal)
+    torch.cuda.synchronize()
+    o_ref, l_ref = orc.fwd(inp.q, inp.k, inp.v, causal=causal)
+    assert max_abs(o.cpu().double().numpy(), o_ref) <= TOL_O_BF16
+    assert max_abs(lse.cpu().double().numpy(), l_ref) <= TOL_LSE_BF16
