@@ -21,10 +21,10 @@
 // TMEM columns: [0,128) S^T (then P^T as bf16 pairs in [0,64)),
 //   [128,256) dP^T (then the dQ tile), [256,256+D) dV, [256+D,256+2D) dK.
 // Per step (query head h, query tile i):
-//   MMA   S^T = K_j Q_i^T,  dP^T = V_j dO_i^T
+//   MMA   S^T = K_j Q_i^T;  dP^T = V_j dO_i^T (once the previous dQ left TMEM)
 //   WG0   P^T = 2^(scale log2e S^T + log2e B^T - log2e LSE) -> TMEM (bf16);
 //         dS^T = P^T o (dP^T - D) -> shared memory (bf16, 128B-swizzled)
-//   MMA   dV += P^T dO_i (P^T from TMEM), dK += dS^T Q_i, dQ_i = dS K_j
+//   MMA   dK += dS^T Q_i and dQ_i = dS K_j, then dV += P^T dO_i (P^T from TMEM)
 //   WG1   dQ_i -> shared memory -> TMA bulk reduce-add into the fp32 accumulator
 #include <algorithm>
 
@@ -53,7 +53,7 @@ struct BwdSmem {
   alignas(16) float nlse2[NSTQ][BM];        // -log2(e) * LSE of the step's query rows (-inf: no key)
   alignas(16) float drow[NSTQ][BM];         // D_i of the step's query rows
   uint64_t kv_full, q_full[NSTQ], q_empty[NSTQ];
-  uint64_t s_full, ds_ready, dq_full, dq_drained, drain;
+  uint64_t st_full, dpt_full, ds_ready, dkq_done, tmem_free, staging_free, drain;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -98,39 +98,35 @@ ATTN_DEVINL void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
   asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
 }
 
-// P^T and dS^T for one key row (this thread) and 128 queries, 32 at a time:
-//   P^T = 2^(scale log2e s + log2e B - log2e LSE), dS^T = P^T (dP^T - D);
-// P^T goes back into TMEM (bf16 pairs, A operand of dV += P^T dO) and dS^T
-// into the 128B-swizzled shared tile.  MASK zeroes queries this key is hidden
-// from (causal: query i sees key j iff j <= i + diag; padding rows and keys).
+// Phase A -- P^T for one key row (this thread) and 128 queries, 32 at a time:
+//   P^T = 2^(scale log2e s + log2e B - log2e LSE), written back into TMEM as
+// bf16 pairs over the S^T columns already read (A operand of dV += P^T dO).
+// MASK zeroes queries this key is hidden from (causal: query i sees key j iff
+// j <= i + diag; padding rows and keys).  Rolled over chunks so the code stays
+// small enough for the instruction cache.
 template <bool MASK, bool HAS_BIAS>
-ATTN_DEVINL void bwd_chunks(uint32_t st_col, uint32_t dp_col, const float* nlse2, const float* drow, uint32_t ds_row,
-                            int r, float scale_log2, const float* bcol, int nk, int i0, int len_q, int kj, int len_k,
-                            int diag) {
+ATTN_DEVINL void bwd_p_chunks(uint32_t st_col, const float* nlse2, float scale_log2, const float* bcol, int nk, int i0,
+                              int len_q, int kj, int len_k, int diag) {
 #pragma unroll 1
   for (int c = 0; c < BM / 32; ++c) {
-    uint32_t sr[32], dpr[32];
+    uint32_t sr[32];
     tmem_ld32(st_col + c * 32, sr);
-    tmem_ld32(dp_col + c * 32, dpr);
     tmem_wait_ld();
     reg_fence(sr);
-    reg_fence(dpr);
     const float4* nl4 = reinterpret_cast<const float4*>(nlse2 + c * 32);
-    const float4* dr4 = reinterpret_cast<const float4*>(drow + c * 32);
-    // queries q0 + e with e < vis are visible from this key
     const int q0 = i0 + c * 32;
-    int vis_lo = 0, vis_hi = 32;
+    int vis_lo = 0, vis_hi = 32;  // queries q0 + e, vis_lo <= e < vis_hi, see this key
     if constexpr (MASK) {
-      vis_lo = kj - diag - q0;                 // causal: q >= kj - diag
-      vis_hi = min(32, len_q - q0);            // padding queries
-      if (kj >= len_k) vis_hi = 0;             // padding key
+      vis_lo = kj - diag - q0;
+      vis_hi = min(32, len_q - q0);
+      if (kj >= len_k) vis_hi = 0;
     }
-    uint32_t pk[16], dk[16];
+    uint32_t pk[16];
 #pragma unroll
     for (int e4 = 0; e4 < 8; ++e4) {
-      const float4 nl = nl4[e4], dr = dr4[e4];
-      const float nlv[4] = {nl.x, nl.y, nl.z, nl.w}, drv[4] = {dr.x, dr.y, dr.z, dr.w};
-      float pv[4], dsv[4];
+      const float4 nl = nl4[e4];
+      const float nlv[4] = {nl.x, nl.y, nl.z, nl.w};
+      float pv[4];
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         const int e = e4 * 4 + u;
@@ -139,16 +135,43 @@ ATTN_DEVINL void bwd_chunks(uint32_t st_col, uint32_t dp_col, const float* nlse2
         float pe = ex2(t);
         if constexpr (MASK) pe = (e >= vis_lo && e < vis_hi) ? pe : 0.f;
         pv[u] = pe;
-        dsv[u] = pe * (__uint_as_float(dpr[e]) - drv[u]);
       }
       pk[2 * e4] = pack_bf16(pv[0], pv[1]);
       pk[2 * e4 + 1] = pack_bf16(pv[2], pv[3]);
+    }
+    tmem_st16(st_col + c * 16, pk);  // columns [16c, 16c+16): S^T there is already read
+  }
+}
+
+// Phase B -- dS^T = P^T (dP^T - D) from the bf16 P^T in TMEM and dP^T, into the
+// 128B-swizzled shared tile (K-major for dK += dS^T Q, MN-major for dQ = dS K).
+ATTN_DEVINL void bwd_ds_chunks(uint32_t st_col, uint32_t dp_col, const float* drow, uint32_t ds_row, int r) {
+#pragma unroll 1
+  for (int c = 0; c < BM / 32; ++c) {
+    uint32_t pr[16], dpr[32];
+    tmem_ld16(st_col + c * 16, pr);
+    tmem_ld32(dp_col + c * 32, dpr);
+    tmem_wait_ld();
+    reg_fence(pr);
+    reg_fence(dpr);
+    const float4* dr4 = reinterpret_cast<const float4*>(drow + c * 32);
+    uint32_t dk[16];
+#pragma unroll
+    for (int e4 = 0; e4 < 8; ++e4) {
+      const float4 dr = dr4[e4];
+      const float drv[4] = {dr.x, dr.y, dr.z, dr.w};
+      float dsv[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int e = e4 * 4 + u;
+        const uint32_t pair = pr[e >> 1];
+        const float pe = __uint_as_float((e & 1) ? (pair & 0xffff0000u) : (pair << 16));
+        dsv[u] = pe * (__uint_as_float(dpr[e]) - drv[u]);
+      }
       dk[2 * e4] = pack_bf16(dsv[0], dsv[1]);
       dk[2 * e4 + 1] = pack_bf16(dsv[2], dsv[3]);
     }
-    // P^T columns [16c, 16c+16) lie in S^T columns already read
-    tmem_st16(st_col + c * 16, pk);
-    // dS^T: 32 queries = 4 chunks of 16 bytes in 64-column block c/2
+    // 32 queries = 4 chunks of 16 bytes in 64-column block c/2
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int chunk = (c & 1) * 4 + u;  // 16-byte chunk within the 128-byte row
@@ -195,10 +218,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&s.q_full[i], 1 + 32);  // TMA transaction arrive + 32 producer lanes (LSE/D rows)
       mbar_init(&s.q_empty[i], 1);
     }
-    mbar_init(&s.s_full, 1);
+    mbar_init(&s.st_full, 1);
+    mbar_init(&s.dpt_full, 1);
     mbar_init(&s.ds_ready, 4);
-    mbar_init(&s.dq_full, 1);
-    mbar_init(&s.dq_drained, 4);
+    mbar_init(&s.dkq_done, 1);
+    mbar_init(&s.tmem_free, 4);
+    mbar_init(&s.staging_free, 1);
     mbar_init(&s.drain, 1);
     fence_mbar_init();
   }
@@ -274,37 +299,46 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int step = 0; ok && step < n_steps; ++step) {
         const int st = step % NSTQ;
         if (!mbar_wait(&s.q_full[st], (step / NSTQ) & 1, ab)) break;
-        // dQ of the previous step must have left TMEM (it lives where dP^T goes);
-        // its commit also covers every earlier MMA, so P^T in S^T's columns is free
-        if (step > 0 && !mbar_wait(&s.dq_drained, (step - 1) & 1, ab)) break;
         tc_fence_after();
         const uint32_t q_addr = smem_u32(s.q[st]), do_addr = smem_u32(s.dout[st]);
-        // S^T = K_j Q_i^T and dP^T = V_j dO_i^T, interleaved (independent accumulators)
+        // S^T = K_j Q_i^T.  It overwrites P^T of the previous step, whose dV MMA
+        // was issued earlier by this thread (tcgen05.mma executes in issue order).
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
           mma_ss(tmem + kColST, sdesc_sw128(k_addr + off, 16, 1024), sdesc_sw128(q_addr + off, 16, 1024), idesc_s,
                  kk > 0);
+        }
+        mma_commit(&s.st_full);
+        // dP^T = V_j dO_i^T goes where dQ of the previous step was
+        if (step > 0 && !mbar_wait(&s.tmem_free, (step - 1) & 1, ab)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
           mma_ss(tmem + kColDPT, sdesc_sw128(v_addr + off, 16, 1024), sdesc_sw128(do_addr + off, 16, 1024),
                  idesc_s, kk > 0);
         }
-        mma_commit(&s.s_full);
+        mma_commit(&s.dpt_full);
         if (!mbar_wait(&s.ds_ready, step & 1, ab)) break;
         tc_fence_after();
-        // dV += P^T dO_i (P^T from TMEM), dK += dS^T Q_i, dQ_i = dS K_j (dS^T read
-        // MN-major): three accumulators, issued round-robin
+        // dK += dS^T Q_i and dQ_i = dS K_j (the dS^T tile read MN-major), issued
+        // round-robin; their commit releases the dS^T tile to the dQ drain
 #pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk) {
           const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
-          mma_ts(tmem + kColDV, tmem + kColST + kk * 8, sdesc_sw128(do_addr + kk * 2048, BM * 128, 1024), idesc_kv,
-                 (step > 0 || kk > 0));
           mma_ss(tmem + kColDK, sdesc_sw128(ds_addr + off, 16, 1024), sdesc_sw128(q_addr + kk * 2048, BM * 128, 1024),
                  idesc_kv, (step > 0 || kk > 0));
           mma_ss(tmem + kColDPT, sdesc_sw128(ds_addr + kk * 2048, 128 * 128, 1024),
                  sdesc_sw128(k_addr + kk * 2048, BN * 128, 1024), idesc_dq, kk > 0);
         }
+        mma_commit(&s.dkq_done);
+        // dV += P^T dO_i (P^T from TMEM)
+#pragma unroll
+        for (int kk = 0; kk < BM / 16; ++kk)
+          mma_ts(tmem + kColDV, tmem + kColST + kk * 8, sdesc_sw128(do_addr + kk * 2048, BM * 128, 1024), idesc_kv,
+                 (step > 0 || kk > 0));
         mma_commit(&s.q_empty[st]);
-        mma_commit(&s.dq_full);
       }
       mma_commit(&s.drain);
       mbar_wait_drain(&s.drain, 0, p.wait_limit);
@@ -321,33 +355,36 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int st = step % NSTQ;
       const int h = hk * G + step / per_head;
       const int i0 = (i_first + step % per_head) * BM;
-      ok = __all_sync(0xffffffffu, mbar_wait(&s.s_full, step & 1, ab));
+      ok = __all_sync(0xffffffffu, mbar_wait(&s.st_full, step & 1, ab));
       if (!ok) break;
-      // q_full for this stage completed before s_full (the MMA waited on it)
+      // q_full for this stage (LSE/D rows) completed before st_full
       tc_fence_after();
-      // tile-level (warp-uniform) condition: the two chunk variants hold
+      // tile-level (warp-uniform) condition: the chunk routines hold
       // warp-collective tcgen05 instructions, so every lane must take the same one
       const bool need_mask = (n0 + BN > len_k) || (i0 + BM > len_q) || (p.causal && n0 + BN - 1 > i0 + diag);
       const float* bcol = nullptr;
       if constexpr (HAS_BIAS) bcol = p.bias + b * p.bias_bstride + (long long)h * p.Nq * p.Nk + min(kj, len_k - 1);
-      // 32 queries per pass; a rolled loop keeps the code small enough for the
-      // instruction cache, and the masked variant is chosen once per step so the
-      // element loop has no branches
       const uint32_t st_col = tmem + lane_off + kColST, dp_col = tmem + lane_off + kColDPT;
       if (need_mask)
-        bwd_chunks<true, HAS_BIAS>(st_col, dp_col, s.nlse2[st], s.drow[st], ds_row, r, p.scale_log2, bcol, p.Nk, i0,
-                                   len_q, kj, len_k, p.causal ? diag : (1 << 30));
+        bwd_p_chunks<true, HAS_BIAS>(st_col, s.nlse2[st], p.scale_log2, bcol, p.Nk, i0, len_q, kj, len_k,
+                                     p.causal ? diag : (1 << 30));
       else
-        bwd_chunks<false, HAS_BIAS>(st_col, dp_col, s.nlse2[st], s.drow[st], ds_row, r, p.scale_log2, bcol, p.Nk, i0,
-                                    len_q, kj, len_k, 1 << 30);
+        bwd_p_chunks<false, HAS_BIAS>(st_col, s.nlse2[st], p.scale_log2, bcol, p.Nk, i0, len_q, kj, len_k, 1 << 30);
       tmem_wait_st();
+      // dS^T needs dP^T, and the shared tile back from the previous dQ drain
+      ok = __all_sync(0xffffffffu, mbar_wait(&s.dpt_full, step & 1, ab) &&
+                                       (step == 0 || mbar_wait(&s.staging_free, (step - 1) & 1, ab)));
+      if (!ok) break;
+      tc_fence_after();
+      bwd_ds_chunks(st_col, dp_col, s.drow[st], ds_row, r);
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s.ds_ready);
     }
     // ---- epilogue: dK (scaled) and dV for this thread's key row
-    if (ok && n_steps > 0) ok = __all_sync(0xffffffffu, mbar_wait(&s.dq_full, (n_steps - 1) & 1, ab));
+    // the MMA warp commits `drain` after its last MMA
+    if (ok && n_steps > 0) ok = __all_sync(0xffffffffu, mbar_wait(&s.drain, 0, ab));
     tc_fence_after();
     if (ok) {
       const long long row = (((long long)b * p.Nk + kj) * p.Hkv + hk) * D;
@@ -381,8 +418,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ===================================================== dQ drain (thread = query row)
-    // dQ_i leaves TMEM through the (now idle) dS^T shared tile, 64 columns per
-    // pass, and is added to the fp32 accumulator by TMA bulk reductions.
+    // dQ_i is read out of TMEM at once (freeing its columns for the next dP^T),
+    // staged through the dS^T shared tile, 64 columns per pass, and added to the
+    // fp32 accumulator by TMA bulk reductions that overlap the next step.
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
@@ -391,27 +429,31 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int step = 0; step < n_steps; ++step) {
       const int h = hk * G + step / per_head;
       const int i0 = (i_first + step % per_head) * BM;
-      if (!__all_sync(0xffffffffu, mbar_wait(&s.dq_full, step & 1, ab))) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(&s.dkq_done, step & 1, ab))) break;
       tc_fence_after();
-#pragma unroll 1
+      uint32_t a[D];
+#pragma unroll
+      for (int c = 0; c < D / 32; ++c) tmem_ld32(tmem + lane_off + kColDPT + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&a[c * 32]));
+      tmem_wait_ld();
+      reg_fence(a);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.tmem_free);
+#pragma unroll
       for (int pass = 0; pass < D / 64; ++pass) {
         if (pass > 0) {
           if (leader) bulk_wait_read0();  // the previous pass's reductions have read the tile
           __syncwarp();
           named_bar_sync(1, 128);
         }
+        // 2 x 32 fp32 = 2 x 8 chunks of 16 bytes, 128B-swizzled like the TMA box
 #pragma unroll
-        for (int cc = 0; cc < 2; ++cc) {
-          uint32_t a[32];
-          tmem_ld32(tmem + lane_off + kColDPT + (pass * 2 + cc) * 32, a);
-          tmem_wait_ld();
-          reg_fence(a);
-          // 32 fp32 = 8 chunks of 16 bytes, 128B-swizzled like the TMA box
+        for (int cc = 0; cc < 2; ++cc)
 #pragma unroll
-          for (int u = 0; u < 8; ++u)
-            st_shared_v4(stage_row + cc * (128 * 128) + ((u ^ (r & 7)) << 4), a[4 * u], a[4 * u + 1], a[4 * u + 2],
-                         a[4 * u + 3]);
-        }
+          for (int u = 0; u < 8; ++u) {
+            const int e = (pass * 2 + cc) * 32 + 4 * u;
+            st_shared_v4(stage_row + cc * (128 * 128) + ((u ^ (r & 7)) << 4), a[e], a[e + 1], a[e + 2], a[e + 3]);
+          }
         fence_proxy_async_smem();
         named_bar_sync(1, 128);
         if (leader) {
@@ -422,11 +464,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         __syncwarp();
       }
-      // the next step's dS^T overwrites the staging tile: wait until it was read
-      if (leader) bulk_wait_read0();
+      // the next step's dS^T overwrites the staging tile: hand it back once read
+      if (leader) {
+        bulk_wait_read0();
+        mbar_arrive(&s.staging_free);
+      }
       __syncwarp();
-      tc_fence_before();
-      if (lane == 0) mbar_arrive(&s.dq_drained);
     }
     if (leader) bulk_wait0();
   }
