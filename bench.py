@@ -36,6 +36,7 @@ METRIC = "attention fwd / fwd+bwd TFLOP/s, causal bf16 N=8192 d=128; % of BF16 p
 SPEC_BF16_TFLOPS = 2250.0
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 TRAFFIC_FILE = ROOT / "profiles" / "bwd_main_causal_b2h32n8192d128_traffic.txt"
+NAIVE_FILE = ROOT / "profiles" / "naive_vs_fused_causal_b1h16n8192d128_bytes.txt"
 BWD_SOURCE = ROOT / "exact_io_aware_57_b200" / "csrc" / "bwd_sm100.cu"
 
 
@@ -51,6 +52,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip timing the CPU oracle")
     ap.add_argument("--batch", type=int, default=None, help="override the batch (profiling a smaller case)")
     ap.add_argument("--heads", type=int, default=None, help="override the head count (profiling a smaller case)")
+    ap.add_argument("--naive", action="store_true",
+                    help="time the fused forward against the materialising three-kernel comparator instead")
     return ap.parse_args(argv)
 
 
@@ -118,6 +121,28 @@ def recorded_traffic():
         return None
     try:
         return int(kv["dram_bytes_per_full_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+def recorded_naive_ratio():
+    """DRAM-bytes ratio (materialising comparator / fused forward) from the
+    committed ncu record, or None if absent or if either source changed."""
+    if not NAIVE_FILE.exists():
+        return None
+    kv = {}
+    for line in NAIVE_FILE.read_text().splitlines():
+        if ":" in line and not line.startswith("#"):
+            k, v = line.split(":", 1)
+            kv[k.strip()] = v.strip()
+    csrc = ROOT / "exact_io_aware_57_b200" / "csrc"
+    if (kv.get("fwd_source_sha256_16") != source_digest(csrc / "fwd_sm100.cu")
+            or kv.get("naive_source_sha256_16") != source_digest(csrc / "naive.cu")):
+        return None
+    try:
+        return {"dram_bytes_ratio": float(kv["dram_bytes_ratio"]), "fused_dram_bytes": int(kv["fused_dram_bytes"]),
+                "naive_dram_bytes": int(kv["naive_dram_bytes"]),
+                "workload": "causal B1 H16 N8192 d128 forward (ncu, same inputs)"}
     except (KeyError, ValueError):
         return None
 
@@ -228,6 +253,8 @@ def run_ours(args):
     dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
     ws = torch.empty(attn.attn_bwd_workspace_size(B, H, N, d), device=dev, dtype=torch.uint8)
     stream = torch.cuda.current_stream()
+    if args.naive:
+        return run_naive(args, w, q, k, v, o, lse, dist, dev, rank, world)
 
     def step():
         attn.attn_fwd(q, k, v, causal=True, out=o, lse=lse)
@@ -344,10 +371,45 @@ def run_ours(args):
             "fwd_bwd_pct_of_spec_peak": round(100 * value / world / SPEC_BF16_TFLOPS, 2),
             "fwd_bwd_pct_of_measured_peak": round(
                 100 * value / world / float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])), 2),
-            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e, "gpu_launches": int(launches),
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "naive_comparator": recorded_naive_ratio(), "gpu_launches": int(launches),
             "gpu_launches_per_step": round(launches / K, 2), "clocks": clk,
         }
         print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+def run_naive(args, w, q, k, v, o, lse, dist, dev, rank, world):
+    """Fused forward vs the materialising comparator (S fp32 -> P bf16 -> PV) on
+    the same inputs: CUDA-event times, and the byte record from the ncu capture
+    of this same command (profiles/), if it matches the current sources."""
+    import torch
+
+    from exact_io_aware_57_b200 import attn
+
+    scratch = torch.empty(attn.attn_naive_scratch_size(w.n, w.n), device=dev, dtype=torch.uint8)
+
+    def timed(fn):
+        for _ in range(args.warmup):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        for _ in range(args.steps):
+            fn()
+        b.record()
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / max(1, args.steps)
+
+    fused = timed(lambda: attn.attn_fwd(q, k, v, causal=True, out=o, lse=lse))
+    naive = timed(lambda: attn.attn_fwd_naive(q, k, v, causal=True, scratch=scratch))
+    if rank == 0:
+        print(json.dumps({"mode": "naive-comparator", "config": {"workload": w.name, "batch": w.batch,
+                                                                 "heads": w.h_q, "seq_len": w.n, "head_dim": w.d},
+                          "fused_fwd_ms": round(fused, 4), "naive_fwd_ms": round(naive, 4),
+                          "naive_scratch_bytes": scratch.numel(), "steps": args.steps, "warmup": args.warmup}),
+              flush=True)
     if dist is not None:
         dist.destroy_process_group()
 
