@@ -50,6 +50,8 @@ def parse_args(argv=None):
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip timing the CPU oracle")
+    ap.add_argument("--workload", default="c3", choices=["c1", "c2", "c3", "c4", "c5a", "c5b"],
+                    help="c3 (default) is the headline causal fwd+bwd workload; the others are reported too")
     ap.add_argument("--batch", type=int, default=None, help="override the batch (profiling a smaller case)")
     ap.add_argument("--heads", type=int, default=None, help="override the head count (profiling a smaller case)")
     ap.add_argument("--naive", action="store_true",
@@ -229,39 +231,93 @@ def plan_oracle_sample(target_s: float):
 
 
 # ------------------------------------------------------------------ our arm
-def run_ours(args):
+def make_job(w, args, dev, rank):
+    """Inputs (pinned host copies + device tensors) and the step of workload w:
+    the forward, plus the backward when the workload trains."""
+    import types
+
     import torch
 
-    from exact_io_aware_57_b200 import attn, synth, workloads
+    from exact_io_aware_57_b200 import attn, synth
+
+    dtype = torch.float32 if w.dtype == "f32" else torch.bfloat16
+    seed = rank_seed(args.seed, rank)
+    j = types.SimpleNamespace(w=w, lengths=None)
+    if w.varlen:
+        j.lengths = synth.varlen_lengths(w.num_seqs, w.len_lo, w.len_hi, seed=args.seed)
+        inp = synth.make_packed(j.lengths, w.h_q, w.h_kv, w.d, dtype=dtype, seed=seed)
+        j.host = {"q": inp.q.pin_memory(), "k": inp.k.pin_memory(), "v": inp.v.pin_memory()}
+        j.dev = {n: t.to(dev) for n, t in j.host.items()}
+        cu = inp.cu_seqlens.to(dev)
+        mx = int(max(j.lengths))
+        j.out = {"o": torch.empty_like(j.dev["q"]), "lse": torch.empty((w.h_q, inp.q.shape[0]), device=dev)}
+
+        def step():
+            attn.attn_fwd_varlen(j.dev["q"], j.dev["k"], j.dev["v"], cu, cu, mx, mx, causal=w.causal,
+                                 out=j.out["o"], lse=j.out["lse"])
+    else:
+        inp = synth.make_dense(w.batch, w.h_q, w.h_kv, w.n, w.n, w.d, dtype=dtype, sigma_qk=w.sigma_qk, seed=seed,
+                               with_dout=w.backward)
+        names = ("q", "k", "v", "dout") if w.backward else ("q", "k", "v")
+        j.host = {n: getattr(inp, n).pin_memory() for n in names}
+        if w.bias:
+            j.host["bias"] = synth.alibi_like_bias(w.h_q, w.n, w.n).pin_memory()
+        j.dev = {n: t.to(dev) for n, t in j.host.items()}
+        j.out = {"o": torch.empty_like(j.dev["q"]), "lse": torch.empty((w.batch, w.h_q, w.n), device=dev)}
+        ws = None
+        if w.backward:
+            j.out.update(dq=torch.empty_like(j.dev["q"]), dk=torch.empty_like(j.dev["k"]),
+                         dv=torch.empty_like(j.dev["v"]))
+            ws = torch.empty(attn.attn_bwd_workspace_size(w.batch, w.h_q, w.n, w.d), device=dev, dtype=torch.uint8)
+
+        def step():
+            d_, o_ = j.dev, j.out
+            attn.attn_fwd(d_["q"], d_["k"], d_["v"], bias=d_.get("bias"), causal=w.causal, out=o_["o"], lse=o_["lse"])
+            if w.backward:
+                attn.attn_bwd(d_["q"], d_["k"], d_["v"], o_["o"], o_["lse"], d_["dout"], bias=d_.get("bias"),
+                              causal=w.causal, workspace=ws, dq=o_["dq"], dk=o_["dk"], dv=o_["dv"])
+    j.step = step
+    j.out_host = {n: torch.empty(t.shape, dtype=t.dtype).pin_memory() for n, t in j.out.items()}
+
+    def e2e_step():
+        for n, t in j.host.items():
+            j.dev[n].copy_(t, non_blocking=True)
+        j.step()
+        for n, t in j.out.items():
+            j.out_host[n].copy_(t, non_blocking=True)
+
+    j.e2e_step = e2e_step
+    j.h2d = sum(t.numel() * t.element_size() for t in j.host.values())
+    j.d2h = sum(t.numel() * t.element_size() for t in j.out.values())
+    j.in_bytes = sum(t.numel() * t.element_size() for t in j.dev.values())
+    return j
+
+
+def run_ours(args):
+    import dataclasses
+
+    import torch
+
+    from exact_io_aware_57_b200 import attn, workloads
 
     rank, world, local = dist_env()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     dist = init_dist(world, "nccl")
-    w = workloads.WORKLOADS["c3"]
+    w = workloads.WORKLOADS[args.workload]
     if args.batch or args.heads:
-        import dataclasses
-
         w = dataclasses.replace(w, name=w.name + " (reduced for profiling)", batch=args.batch or w.batch,
                                 h_q=args.heads or w.h_q, h_kv=args.heads or w.h_kv)
-    B, H, N, d = w.batch, w.h_q, w.n, w.d
-    inp = synth.make_dense(B, H, H, N, N, d, sigma_qk=w.sigma_qk, seed=rank_seed(args.seed, rank))
-    host = {n: getattr(inp, n).pin_memory() for n in ("q", "k", "v", "dout")}
-    q, k, v, do = (host[n].to(dev) for n in ("q", "k", "v", "dout"))
-    o = torch.empty_like(q)
-    lse = torch.empty((B, H, N), device=dev, dtype=torch.float32)
-    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
-    ws = torch.empty(attn.attn_bwd_workspace_size(B, H, N, d), device=dev, dtype=torch.uint8)
-    stream = torch.cuda.current_stream()
     if args.naive:
-        return run_naive(args, w, q, k, v, o, lse, dist, dev, rank, world)
-
-    def step():
-        attn.attn_fwd(q, k, v, causal=True, out=o, lse=lse)
-        attn.attn_bwd(q, k, v, o, lse, do, causal=True, workspace=ws, dq=dq, dk=dk, dv=dv)
+        job = make_job(dataclasses.replace(w, backward=False, bias=False), args, dev, rank)
+        return run_naive(args, w, job.dev["q"], job.dev["k"], job.dev["v"], job.out["o"], job.out["lse"], dist, dev,
+                         rank, world)
+    job = make_job(w, args, dev, rank)
+    stream = torch.cuda.current_stream()
+    tensor_path = w.dtype != "f32"
 
     for _ in range(args.warmup):
-        step()
+        job.step()
     torch.cuda.synchronize()
     if attn.attn_device_status() != 0:
         raise RuntimeError("device status reported a timeout during warm-up")
@@ -282,7 +338,7 @@ def run_ours(args):
     for i in range(K):
         attn.attn_set_kernel_events(attn.ATTN_KERNEL_FWD, *fwd_ev[i])
         attn.attn_set_kernel_events(attn.ATTN_KERNEL_BWD, *bwd_ev[i])
-        step()
+        job.step()
     t_end.record(stream)
     torch.cuda.synchronize()
     launches = attn.attn_launch_count(reset=True)
@@ -295,85 +351,82 @@ def run_ours(args):
 
     ms_total = max_over_ranks(dist, t_start.elapsed_time(t_end), dev)
     ms_step = ms_total / K
-    fwd_ms = statistics.mean(a.elapsed_time(b) for a, b in fwd_ev)
-    bwd_main_ms = statistics.mean(a.elapsed_time(b) for a, b in bwd_ev)
-    fwd_ms = max_over_ranks(dist, fwd_ms, dev)
-    bwd_main_ms = max_over_ranks(dist, bwd_main_ms, dev)
-    f_fwd = workloads.flops(w, backward=False)
-    f_step = workloads.flops(w, backward=True)
+    fwd_ms = bwd_main_ms = None
+    if tensor_path:
+        fwd_ms = max_over_ranks(dist, statistics.mean(a.elapsed_time(b) for a, b in fwd_ev), dev)
+        if w.backward:
+            bwd_main_ms = max_over_ranks(dist, statistics.mean(a.elapsed_time(b) for a, b in bwd_ev), dev)
+    f_fwd = workloads.flops(w, backward=False, lengths=job.lengths)
+    f_step = workloads.flops(w, lengths=job.lengths)
     value = world * f_step / (ms_step * 1e-3) / 1e12
 
     # ---- end to end through the public API with pinned host buffers
     e2e = None
     if not args.no_e2e:
-        out_host = {"o": torch.empty_like(host["q"]).pin_memory(), "lse": torch.empty((B, H, N)).pin_memory(),
-                    "dq": torch.empty_like(host["q"]).pin_memory(), "dk": torch.empty_like(host["k"]).pin_memory(),
-                    "dv": torch.empty_like(host["v"]).pin_memory()}
-
-        def e2e_step():
-            q.copy_(host["q"], non_blocking=True)
-            k.copy_(host["k"], non_blocking=True)
-            v.copy_(host["v"], non_blocking=True)
-            do.copy_(host["dout"], non_blocking=True)
-            step()
-            out_host["o"].copy_(o, non_blocking=True)
-            out_host["lse"].copy_(lse, non_blocking=True)
-            out_host["dq"].copy_(dq, non_blocking=True)
-            out_host["dk"].copy_(dk, non_blocking=True)
-            out_host["dv"].copy_(dv, non_blocking=True)
-
         ke = max(3, K // 10)
         for _ in range(2):
-            e2e_step()
+            job.e2e_step()
         barrier(dist, local)
         torch.cuda.synchronize()
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         for _ in range(ke):
-            e2e_step()
+            job.e2e_step()
         b.record(stream)
         torch.cuda.synchronize()
         barrier(dist, local)
         e2e_ms = max_over_ranks(dist, a.elapsed_time(b) / ke, dev)
-        h2d = sum(host[n].numel() * host[n].element_size() for n in ("q", "k", "v", "dout"))
-        d2h = sum(t.numel() * t.element_size() for t in out_host.values())
-        e2e = {"value": round(world * f_step / (e2e_ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
-               "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(d2h)}
+        e2e = {"value": round(world * f_step / (e2e_ms * 1e-3) / 1e12, 4), "unit": "TFLOP/s",
+               "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": int(job.h2d), "d2h_bytes_per_step": int(job.d2h)}
 
     peaks, peak_kind = measured_peaks()
-    bwd_flops = 2.5 * f_fwd
-    achieved = bwd_flops / (bwd_main_ms * 1e-3) / 1e12
     peak = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
-    roofline = {"kernel": "bwd_main_kernel<128> (tensor-core backward)", "bound": "tensor",
-                "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s", "frac": round(achieved / peak, 4),
-                "peak_kind": f"bf16 dense, sustained, {peak_kind}", "traffic": recorded_traffic(),
-                "algorithmic_flops_per_launch": bwd_flops, "avg_launch_ms": round(bwd_main_ms, 4)}
+    if not tensor_path:
+        roofline = {"kernel": "fp32 CUDA-core path", "bound": "latency", "achieved": None, "peak": None,
+                    "unit": "TFLOP/s", "frac": None, "traffic": None,
+                    "note": "4-MFLOP problem: bound by launch latency; checked for parity"}
+    else:
+        kern_flops = (2.5 if w.backward else 1.0) * f_fwd
+        kern_ms = bwd_main_ms if w.backward else fwd_ms
+        achieved = kern_flops / (kern_ms * 1e-3) / 1e12
+        headline = args.workload == "c3" and not (args.batch or args.heads)
+        roofline = {"kernel": "bwd_main_kernel (tensor-core backward)" if w.backward
+                    else "fwd_sm100_kernel (tensor-core forward)",
+                    "bound": "tensor", "achieved": round(achieved, 2), "peak": peak, "unit": "TFLOP/s",
+                    "frac": round(achieved / peak, 4), "peak_kind": f"bf16 dense, sustained, {peak_kind}",
+                    "traffic": recorded_traffic() if (w.backward and headline) else None,
+                    "algorithmic_flops_per_launch": kern_flops, "avg_launch_ms": round(kern_ms, 4)}
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and args.workload == "c3":
         prefix, heads = plan_oracle_sample(15.0)
         dt, fl = oracle_sample(prefix, heads, args.seed)
         cpu = {"value": round(fl / dt / 1e12, 6), "unit": "TFLOP/s", "cores": cpu_threads(), "kind": "oracle",
                "sample": f"fp64 oracle fwd+bwd on the causal prefix of {prefix} tokens of {heads} heads "
                          f"(batch element 0, d=128, Q/K std 3), {dt:.1f} s"}
 
+    l2_note = (f"no flush: inputs ({job.in_bytes / 1e6:.0f} MB) exceed the 126 MB L2" if job.in_bytes > 126e6
+               else f"no flush: inputs ({job.in_bytes / 1e6:.1f} MB) fit in L2 (small workload)")
     if rank == 0:
         line = {
-            "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": K,
-            "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic (seeded randn; Q/K std 3, V/dO std 1)",
-            "config": {"workload": w.name, "batch": B, "heads": H, "seq_len": N, "head_dim": d, "causal": True,
-                       "global_batch": B * world, "parallelism": f"dp{world} (independent problem per GPU)",
-                       "l2": "no flush: inputs (4 x 134 MB) and outputs exceed the 126 MB L2"},
-            "fwd_tflops": round(world * f_fwd / (fwd_ms * 1e-3) / 1e12, 2),
-            "fwd_ms": round(fwd_ms, 4),
-            "fwd_pct_of_spec_peak": round(100 * f_fwd / (fwd_ms * 1e-3) / 1e12 / SPEC_BF16_TFLOPS, 2),
-            "fwd_bwd_pct_of_spec_peak": round(100 * value / world / SPEC_BF16_TFLOPS, 2),
-            "fwd_bwd_pct_of_measured_peak": round(
+            "metric": METRIC, "value": round(value, 2 if tensor_path else 6), "unit": "TFLOP/s", "n_gpus": world,
+            "steps": K, "warmup": args.warmup, "ms_per_step": round(ms_step, 4), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+            "data": f"synthetic (seeded randn; Q/K std {w.sigma_qk:g}, V/dO std 1)",
+            "config": {"workload": w.name, "batch": w.batch, "heads": w.h_q, "kv_heads": w.h_kv,
+                       "seq_len": w.n if not w.varlen else f"{w.num_seqs} seqs, {int(sum(job.lengths))} tokens",
+                       "head_dim": w.d, "causal": w.causal, "bias": w.bias, "backward": w.backward,
+                       "global_batch": w.batch * world, "parallelism": f"dp{world} (independent problem per GPU)",
+                       "l2": l2_note},
+            "fwd_tflops": round(world * f_fwd / (fwd_ms * 1e-3) / 1e12, 2) if fwd_ms else None,
+            "fwd_ms": round(fwd_ms, 4) if fwd_ms else None,
+            "fwd_pct_of_spec_peak": round(100 * f_fwd / (fwd_ms * 1e-3) / 1e12 / SPEC_BF16_TFLOPS, 2) if fwd_ms else None,
+            "step_pct_of_spec_peak": round(100 * value / world / SPEC_BF16_TFLOPS, 2),
+            "step_pct_of_measured_peak": round(
                 100 * value / world / float(peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])), 2),
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-            "naive_comparator": recorded_naive_ratio(), "gpu_launches": int(launches),
-            "gpu_launches_per_step": round(launches / K, 2), "clocks": clk,
+            "naive_comparator": recorded_naive_ratio() if args.workload == "c3" else None,
+            "gpu_launches": int(launches), "gpu_launches_per_step": round(launches / K, 2), "clocks": clk,
         }
         print(json.dumps(line), flush=True)
     if dist is not None:
