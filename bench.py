@@ -54,6 +54,8 @@ def parse_args(argv=None):
                     help="c3 (default) is the headline causal fwd+bwd workload; the others are reported too")
     ap.add_argument("--batch", type=int, default=None, help="override the batch (profiling a smaller case)")
     ap.add_argument("--heads", type=int, default=None, help="override the head count (profiling a smaller case)")
+    ap.add_argument("--bias-mode", default="dense", choices=["dense", "alibi"],
+                    help="grouped workload: read the dense fp32 bias tensor, or form it in-kernel from slopes")
     ap.add_argument("--naive", action="store_true",
                     help="time the fused forward against the materialising three-kernel comparator instead")
     return ap.parse_args(argv)
@@ -260,8 +262,11 @@ def make_job(w, args, dev, rank):
                                with_dout=w.backward)
         names = ("q", "k", "v", "dout") if w.backward else ("q", "k", "v")
         j.host = {n: getattr(inp, n).pin_memory() for n in names}
-        if w.bias:
+        if w.bias and args.bias_mode == "dense":
             j.host["bias"] = synth.alibi_like_bias(w.h_q, w.n, w.n).pin_memory()
+        elif w.bias:
+            # the same bias from its per-head slopes, formed inside the kernels
+            j.host["alibi"] = synth.alibi_like_slopes(w.h_q).pin_memory()
         j.dev = {n: t.to(dev) for n, t in j.host.items()}
         j.out = {"o": torch.empty_like(j.dev["q"]), "lse": torch.empty((w.batch, w.h_q, w.n), device=dev)}
         ws = None
@@ -272,10 +277,12 @@ def make_job(w, args, dev, rank):
 
         def step():
             d_, o_ = j.dev, j.out
-            attn.attn_fwd(d_["q"], d_["k"], d_["v"], bias=d_.get("bias"), causal=w.causal, out=o_["o"], lse=o_["lse"])
+            attn.attn_fwd(d_["q"], d_["k"], d_["v"], bias=d_.get("bias"), causal=w.causal, out=o_["o"], lse=o_["lse"],
+                          alibi_slopes=d_.get("alibi"))
             if w.backward:
                 attn.attn_bwd(d_["q"], d_["k"], d_["v"], o_["o"], o_["lse"], d_["dout"], bias=d_.get("bias"),
-                              causal=w.causal, workspace=ws, dq=o_["dq"], dk=o_["dk"], dv=o_["dv"])
+                              causal=w.causal, workspace=ws, dq=o_["dq"], dk=o_["dk"], dv=o_["dv"],
+                              alibi_slopes=d_.get("alibi"))
     j.step = step
     j.out_host = {n: torch.empty(t.shape, dtype=t.dtype).pin_memory() for n, t in j.out.items()}
 
@@ -415,7 +422,9 @@ def run_ours(args):
             "data": f"synthetic (seeded randn; Q/K std {w.sigma_qk:g}, V/dO std 1)",
             "config": {"workload": w.name, "batch": w.batch, "heads": w.h_q, "kv_heads": w.h_kv,
                        "seq_len": w.n if not w.varlen else f"{w.num_seqs} seqs, {int(sum(job.lengths))} tokens",
-                       "head_dim": w.d, "causal": w.causal, "bias": w.bias, "backward": w.backward,
+                       "head_dim": w.d, "causal": w.causal,
+                       "bias": (("dense fp32 tensor" if args.bias_mode == "dense" else "per-head slopes, formed in-kernel")
+                                if w.bias else False), "backward": w.backward,
                        "global_batch": w.batch * world, "parallelism": f"dp{world} (independent problem per GPU)",
                        "l2": l2_note},
             "fwd_tflops": round(world * f_fwd / (fwd_ms * 1e-3) / 1e12, 2) if fwd_ms else None,

@@ -32,6 +32,9 @@ _VP, _FP, _IP = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p
 _I, _LL, _F, _SZ = ctypes.c_int, ctypes.c_longlong, ctypes.c_float, ctypes.c_size_t
 EXPORTS = {
     "attn_fwd": (_I, [_VP, _VP, _VP, _FP, _LL, _VP, _FP, _I, _I, _I, _I, _I, _I, _F, _I, _I, _VP]),
+    "attn_fwd_alibi": (_I, [_VP, _VP, _VP, _FP, _VP, _FP, _I, _I, _I, _I, _I, _I, _F, _I, _I, _VP]),
+    "attn_bwd_alibi": (_I, [_VP, _VP, _VP, _FP, _VP, _FP, _VP, _VP, _VP, _VP, _VP, _SZ, _I, _I, _I, _I, _I, _I,
+                            _F, _I, _I, _VP]),
     "attn_bwd_workspace_size": (_SZ, [_I, _I, _I, _I]),
     "attn_bwd": (_I, [_VP, _VP, _VP, _FP, _LL, _VP, _FP, _VP, _VP, _VP, _VP, _VP, _SZ, _I, _I, _I, _I, _I,
                       _I, _F, _I, _I, _VP]),
@@ -112,13 +115,28 @@ def _bias_args(bias, B, Hq, Nq, Nk):
     raise AttnError("bias must be [Hq,Nq,Nk] or [B,Hq,Nq,Nk]")
 
 
-def attn_fwd(q, k, v, bias=None, causal=False, scale=None, out=None, lse=None, stream=None):
-    """O, LSE = attention(q [B,Nq,Hq,d], k/v [B,Nk,Hkv,d]); o like q, lse fp32 [B,Hq,Nq]."""
+def _slopes(alibi_slopes, Hq):
+    if alibi_slopes.dtype != torch.float32 or alibi_slopes.numel() != Hq:
+        raise AttnError("alibi_slopes must be fp32 [h_q]")
+    return _dev(alibi_slopes, "alibi_slopes")
+
+
+def attn_fwd(q, k, v, bias=None, causal=False, scale=None, out=None, lse=None, stream=None, alibi_slopes=None):
+    """O, LSE = attention(q [B,Nq,Hq,d], k/v [B,Nk,Hkv,d]); o like q, lse fp32 [B,Hq,Nq].
+    bias: dense fp32 [Hq,Nq,Nk] or [B,Hq,Nq,Nk]; alibi_slopes: fp32 [Hq] (bias
+    -slope_h |j - (i + Nk - Nq)| formed in the kernel); at most one of the two."""
     B, Nq, Hq, d = q.shape
     Nk, Hkv = k.shape[1], k.shape[2]
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     o = torch.empty_like(q) if out is None else out
     lse = torch.empty((B, Hq, Nq), device=q.device, dtype=torch.float32) if lse is None else lse
+    if alibi_slopes is not None:
+        if bias is not None:
+            raise AttnError("pass either bias or alibi_slopes")
+        _check(_lib.attn_fwd_alibi(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _slopes(alibi_slopes, Hq),
+                                   _dev(o, "o"), _dev(lse, "lse"), B, Hq, Hkv, Nq, Nk, d, scale, int(bool(causal)),
+                                   _dtype_code(q), _stream(stream)))
+        return o, lse
     bp, bs = _bias_args(bias, B, Hq, Nq, Nk)
     _check(_lib.attn_fwd(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), bp, bs, _dev(o, "o"), _dev(lse, "lse"),
                          B, Hq, Hkv, Nq, Nk, d, scale, int(bool(causal)), _dtype_code(q), _stream(stream)))
@@ -130,7 +148,7 @@ def attn_bwd_workspace_size(batch, h_q, n_q, d) -> int:
 
 
 def attn_bwd(q, k, v, o, lse, dout, bias=None, causal=False, scale=None, workspace=None, dq=None, dk=None,
-             dv=None, stream=None):
+             dv=None, stream=None, alibi_slopes=None):
     """dq, dk, dv of attn_fwd for upstream gradient dout (layouts as q, k, v)."""
     B, Nq, Hq, d = q.shape
     Nk, Hkv = k.shape[1], k.shape[2]
@@ -141,6 +159,15 @@ def attn_bwd(q, k, v, o, lse, dout, bias=None, causal=False, scale=None, workspa
     need = attn_bwd_workspace_size(B, Hq, Nq, d)
     if workspace is None:
         workspace = torch.empty(need, device=q.device, dtype=torch.uint8)
+    if alibi_slopes is not None:
+        if bias is not None:
+            raise AttnError("pass either bias or alibi_slopes")
+        _check(_lib.attn_bwd_alibi(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _slopes(alibi_slopes, Hq),
+                                   _dev(o, "o"), _dev(lse, "lse"), _dev(dout, "dout"), _dev(dq, "dq"),
+                                   _dev(dk, "dk"), _dev(dv, "dv"), _dev(workspace, "workspace"),
+                                   workspace.numel() * workspace.element_size(), B, Hq, Hkv, Nq, Nk, d, scale,
+                                   int(bool(causal)), _dtype_code(q), _stream(stream)))
+        return dq, dk, dv
     bp, bs = _bias_args(bias, B, Hq, Nq, Nk)
     _check(_lib.attn_bwd(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), bp, bs, _dev(o, "o"), _dev(lse, "lse"),
                          _dev(dout, "dout"), _dev(dq, "dq"), _dev(dk, "dk"), _dev(dv, "dv"),

@@ -108,9 +108,13 @@ int check_common(int batch, int h_q, int h_kv, int n_q, int n_k, int d, int dtyp
 
 extern "C" {
 
-int attn_fwd(const void* q, const void* k, const void* v, const float* bias, long long bias_batch_stride, void* o,
-             float* lse, int batch, int h_q, int h_kv, int n_q, int n_k, int d, float scale, int causal, int dtype,
-             void* stream) {
+}  // extern "C"
+
+namespace {
+
+int fwd_impl(const void* q, const void* k, const void* v, const float* bias, long long bias_batch_stride,
+             const float* alibi, void* o, float* lse, int batch, int h_q, int h_kv, int n_q, int n_k, int d,
+             float scale, int causal, int dtype, void* stream) {
   int rc = check_common(batch, h_q, h_kv, n_q, n_k, d, dtype);
   if (rc) return rc;
   if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID;
@@ -124,6 +128,7 @@ int attn_fwd(const void* q, const void* k, const void* v, const float* bias, lon
     p.k = static_cast<const float*>(k);
     p.v = static_cast<const float*>(v);
     p.bias = bias;
+    p.alibi = alibi;
     p.o = static_cast<float*>(o);
     p.lse = lse;
     p.q_bstride = (long long)n_q * h_q * d;
@@ -154,7 +159,27 @@ int attn_fwd(const void* q, const void* k, const void* v, const float* bias, lon
   g.scale = scale;
   g.bias = bias;
   g.bias_bstride = bias_batch_stride;
+  g.alibi = alibi;
   return launch_fwd_sm100(g, static_cast<__nv_bfloat16*>(o), lse, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+int attn_fwd(const void* q, const void* k, const void* v, const float* bias, long long bias_batch_stride, void* o,
+             float* lse, int batch, int h_q, int h_kv, int n_q, int n_k, int d, float scale, int causal, int dtype,
+             void* stream) {
+  return fwd_impl(q, k, v, bias, bias_batch_stride, nullptr, o, lse, batch, h_q, h_kv, n_q, n_k, d, scale, causal,
+                  dtype, stream);
+}
+
+int attn_fwd_alibi(const void* q, const void* k, const void* v, const float* alibi_slopes, void* o, float* lse,
+                   int batch, int h_q, int h_kv, int n_q, int n_k, int d, float scale, int causal, int dtype,
+                   void* stream) {
+  if (!alibi_slopes) return ATTN_ERR_INVALID;
+  return fwd_impl(q, k, v, nullptr, 0, alibi_slopes, o, lse, batch, h_q, h_kv, n_q, n_k, d, scale, causal, dtype,
+                  stream);
 }
 
 size_t attn_bwd_workspace_size(int batch, int h_q, int n_q, int d) {
@@ -162,10 +187,14 @@ size_t attn_bwd_workspace_size(int batch, int h_q, int n_q, int d) {
   return align256((size_t)batch * n_q * h_q * d * sizeof(float)) + align256((size_t)batch * h_q * n_q * sizeof(float));
 }
 
-int attn_bwd(const void* q, const void* k, const void* v, const float* bias, long long bias_batch_stride,
-             const void* o, const float* lse, const void* dout, void* dq, void* dk, void* dv, void* workspace,
-             size_t workspace_bytes, int batch, int h_q, int h_kv, int n_q, int n_k, int d, float scale, int causal,
-             int dtype, void* stream) {
+}  // extern "C"
+
+namespace {
+
+int bwd_impl(const void* q, const void* k, const void* v, const float* bias, long long bias_batch_stride,
+             const float* alibi, const void* o, const float* lse, const void* dout, void* dq, void* dk, void* dv,
+             void* workspace, size_t workspace_bytes, int batch, int h_q, int h_kv, int n_q, int n_k, int d,
+             float scale, int causal, int dtype, void* stream) {
   int rc = check_common(batch, h_q, h_kv, n_q, n_k, d, dtype);
   if (rc) return rc;
   if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return ATTN_ERR_INVALID;
@@ -189,6 +218,7 @@ int attn_bwd(const void* q, const void* k, const void* v, const float* bias, lon
     p.k = static_cast<const float*>(k);
     p.v = static_cast<const float*>(v);
     p.bias = bias;
+    p.alibi = alibi;
     p.lse = const_cast<float*>(lse);
     p.q_bstride = (long long)n_q * h_q * d;
     p.k_bstride = (long long)n_k * h_kv * d;
@@ -219,9 +249,31 @@ int attn_bwd(const void* q, const void* k, const void* v, const float* bias, lon
   g.scale = scale;
   g.bias = bias;
   g.bias_bstride = bias_batch_stride;
+  g.alibi = alibi;
   return launch_bwd_sm100(g, static_cast<const __nv_bfloat16*>(o), lse, static_cast<const __nv_bfloat16*>(dout),
                           static_cast<__nv_bfloat16*>(dq), static_cast<__nv_bfloat16*>(dk),
                           static_cast<__nv_bfloat16*>(dv), dq_acc, Drow, st);
+}
+
+}  // namespace
+
+extern "C" {
+
+int attn_bwd(const void* q, const void* k, const void* v, const float* bias, long long bias_batch_stride,
+             const void* o, const float* lse, const void* dout, void* dq, void* dk, void* dv, void* workspace,
+             size_t workspace_bytes, int batch, int h_q, int h_kv, int n_q, int n_k, int d, float scale, int causal,
+             int dtype, void* stream) {
+  return bwd_impl(q, k, v, bias, bias_batch_stride, nullptr, o, lse, dout, dq, dk, dv, workspace, workspace_bytes,
+                  batch, h_q, h_kv, n_q, n_k, d, scale, causal, dtype, stream);
+}
+
+int attn_bwd_alibi(const void* q, const void* k, const void* v, const float* alibi_slopes, const void* o,
+                   const float* lse, const void* dout, void* dq, void* dk, void* dv, void* workspace,
+                   size_t workspace_bytes, int batch, int h_q, int h_kv, int n_q, int n_k, int d, float scale,
+                   int causal, int dtype, void* stream) {
+  if (!alibi_slopes) return ATTN_ERR_INVALID;
+  return bwd_impl(q, k, v, nullptr, 0, alibi_slopes, o, lse, dout, dq, dk, dv, workspace, workspace_bytes, batch,
+                  h_q, h_kv, n_q, n_k, d, scale, causal, dtype, stream);
 }
 
 int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse, const int* cu_seqlens_q,

@@ -66,6 +66,7 @@ struct BwdParams {
   __nv_bfloat16* dv;
   const float* bias;
   long long bias_bstride;
+  const float* alibi;
   int Hq, Hkv, Nq, Nk;
   float scale, scale_log2;
   int causal;
@@ -104,9 +105,10 @@ ATTN_DEVINL void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
 // MASK zeroes queries this key is hidden from (causal: query i sees key j iff
 // j <= i + diag; padding rows and keys).  Rolled over chunks so the code stays
 // small enough for the instruction cache.
-template <bool MASK, bool HAS_BIAS>
-ATTN_DEVINL void bwd_p_chunks(uint32_t st_col, const float* nlse2, float scale_log2, const float* bcol, int nk, int i0,
-                              int len_q, int kj, int len_k, int diag) {
+template <bool MASK, int BIAS>
+ATTN_DEVINL void bwd_p_chunks(uint32_t st_col, const float* nlse2, float scale_log2, const float* bcol,
+                              float neg_slope2, int nk, int i0, int len_q, int kj, int len_k, int diag,
+                              int bias_diag) {
 #pragma unroll 1
   for (int c = 0; c < BM / 32; ++c) {
     uint32_t sr[32];
@@ -131,7 +133,9 @@ ATTN_DEVINL void bwd_p_chunks(uint32_t st_col, const float* nlse2, float scale_l
       for (int u = 0; u < 4; ++u) {
         const int e = e4 * 4 + u;
         float t = fmaf(__uint_as_float(sr[e]), scale_log2, nlv[u]);
-        if constexpr (HAS_BIAS) t = fmaf(__ldg(bcol + (long long)min(q0 + e, len_q - 1) * nk), kLog2e, t);
+        if constexpr (BIAS == kBiasDense) t = fmaf(__ldg(bcol + (long long)min(q0 + e, len_q - 1) * nk), kLog2e, t);
+        if constexpr (BIAS == kBiasAlibi)
+          t = fmaf(neg_slope2, fabsf(static_cast<float>(kj - q0 - e - bias_diag)), t);
         float pe = ex2(t);
         if constexpr (MASK) pe = (e >= vis_lo && e < vis_hi) ? pe : 0.f;
         pv[u] = pe;
@@ -181,7 +185,7 @@ ATTN_DEVINL void bwd_ds_chunks(uint32_t st_col, uint32_t dp_col, const float* dr
   }
 }
 
-template <int D, bool HAS_BIAS>
+template <int D, int BIAS>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
@@ -363,13 +367,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       // warp-collective tcgen05 instructions, so every lane must take the same one
       const bool need_mask = (n0 + BN > len_k) || (i0 + BM > len_q) || (p.causal && n0 + BN - 1 > i0 + diag);
       const float* bcol = nullptr;
-      if constexpr (HAS_BIAS) bcol = p.bias + b * p.bias_bstride + (long long)h * p.Nq * p.Nk + min(kj, len_k - 1);
+      if constexpr (BIAS == kBiasDense) bcol = p.bias + b * p.bias_bstride + (long long)h * p.Nq * p.Nk + min(kj, len_k - 1);
+      float neg_slope2 = 0.f;
+      if constexpr (BIAS == kBiasAlibi) neg_slope2 = -__ldg(p.alibi + h) * kLog2e;
       const uint32_t st_col = tmem + lane_off + kColST, dp_col = tmem + lane_off + kColDPT;
       if (need_mask)
-        bwd_p_chunks<true, HAS_BIAS>(st_col, s.nlse2[st], p.scale_log2, bcol, p.Nk, i0, len_q, kj, len_k,
-                                     p.causal ? diag : (1 << 30));
+        bwd_p_chunks<true, BIAS>(st_col, s.nlse2[st], p.scale_log2, bcol, neg_slope2, p.Nk, i0, len_q, kj, len_k,
+                                 p.causal ? diag : (1 << 30), diag);
       else
-        bwd_p_chunks<false, HAS_BIAS>(st_col, s.nlse2[st], p.scale_log2, bcol, p.Nk, i0, len_q, kj, len_k, 1 << 30);
+        bwd_p_chunks<false, BIAS>(st_col, s.nlse2[st], p.scale_log2, bcol, neg_slope2, p.Nk, i0, len_q, kj, len_k,
+                                  1 << 30, diag);
       tmem_wait_st();
       // dS^T needs dP^T, and the shared tile back from the previous dQ drain
       ok = __all_sync(0xffffffffu, mbar_wait(&s.dpt_full, step & 1, ab) &&
@@ -521,11 +528,11 @@ __global__ void __launch_bounds__(256) bwd_dq_kernel(const float* __restrict__ a
                                                pack_bf16(c.x * scale, c.y * scale), pack_bf16(c.z * scale, c.w * scale));
 }
 
-template <int D, bool HAS_BIAS>
+template <int D, int BIAS>
 int launch_main_t(const TcGeom& g, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                   const CUtensorMap& mdo, const CUtensorMap& mdq, const BwdParams& p, cudaStream_t st) {
   const size_t smem = std::max<size_t>(sizeof(BwdSmem<D>), 116 * 1024);
-  auto kern = bwd_main_kernel<D, HAS_BIAS>;
+  auto kern = bwd_main_kernel<D, BIAS>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return ATTN_ERR_CUDA;
   dim3 grid((g.Nk + BN - 1) / BN, g.Hkv, g.B);
@@ -581,6 +588,7 @@ int launch_bwd_sm100(const TcGeom& g, const __nv_bfloat16* o, const float* lse, 
   p.dv = dv;
   p.bias = g.bias;
   p.bias_bstride = g.bias_bstride;
+  p.alibi = g.alibi;
   p.Hq = g.Hq;
   p.Hkv = g.Hkv;
   p.Nq = g.Nq;
@@ -592,12 +600,14 @@ int launch_bwd_sm100(const TcGeom& g, const __nv_bfloat16* o, const float* lse, 
   p.wait_limit = kWaitLimitCycles;
   if (!p.status) return ATTN_ERR_CUDA;
   int rc;
-  const bool hb = g.bias != nullptr;
   if (g.D == 64)
-    rc = hb ? launch_main_t<64, true>(g, mq, mk, mv, mdo, mdq, p, st) : launch_main_t<64, false>(g, mq, mk, mv, mdo, mdq, p, st);
+    rc = g.bias    ? launch_main_t<64, kBiasDense>(g, mq, mk, mv, mdo, mdq, p, st)
+         : g.alibi ? launch_main_t<64, kBiasAlibi>(g, mq, mk, mv, mdo, mdq, p, st)
+                   : launch_main_t<64, kBiasNone>(g, mq, mk, mv, mdo, mdq, p, st);
   else
-    rc = hb ? launch_main_t<128, true>(g, mq, mk, mv, mdo, mdq, p, st)
-            : launch_main_t<128, false>(g, mq, mk, mv, mdo, mdq, p, st);
+    rc = g.bias    ? launch_main_t<128, kBiasDense>(g, mq, mk, mv, mdo, mdq, p, st)
+         : g.alibi ? launch_main_t<128, kBiasAlibi>(g, mq, mk, mv, mdo, mdq, p, st)
+                   : launch_main_t<128, kBiasNone>(g, mq, mk, mv, mdo, mdq, p, st);
   if (rc) return rc;
   // 3) dQ
   const long long n8 = (long long)g.B * g.Nq * g.Hq * g.D / 8;

@@ -234,6 +234,10 @@ ATTN_DEVINL uint32_t pack_bf16(float lo, float hi) {
 }
 
 constexpr float kLog2e = 1.4426950408889634f;
+
+// Additive score bias variants: none, a dense fp32 tensor, or ALiBi slopes
+// (B[h, i, j] = -slope_h |j - (i + n_k - n_q)|, formed in registers).
+constexpr int kBiasNone = 0, kBiasDense = 1, kBiasAlibi = 2;
 constexpr float kLn2 = 0.6931471805599453f;
 
 }  // namespace attn

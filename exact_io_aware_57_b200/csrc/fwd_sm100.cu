@@ -60,6 +60,7 @@ struct FwdParams {
   float* lse;
   const float* bias;
   long long bias_bstride;
+  const float* alibi;  // per-query-head slopes (BIAS == kBiasAlibi)
   const int* cu_q;
   const int* cu_k;
   int Hq, Hkv, Nq, Nk;
@@ -77,7 +78,7 @@ ATTN_DEVINL void reg_fence(uint32_t (&r)[N]) {
   for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
 }
 
-template <int D, bool HAS_BIAS, bool FAST>
+template <int D, int BIAS, bool FAST>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -234,7 +235,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool row_ok = i < len_q;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const float* brow = nullptr;  // rows past the end read the last row (their output is dropped)
-    if constexpr (HAS_BIAS) brow = p.bias + bidx * p.bias_bstride + ((long long)h * p.Nq + min(i, len_q - 1)) * p.Nk;
+    if constexpr (BIAS == kBiasDense)
+      brow = p.bias + bidx * p.bias_bstride + ((long long)h * p.Nq + min(i, len_q - 1)) * p.Nk;
+    float neg_slope2 = 0.f;  // ALiBi: B = -slope |key - (i + diag)|, in log2 units
+    if constexpr (BIAS == kBiasAlibi) neg_slope2 = -__ldg(p.alibi + h) * kLog2e;
     // m: the reference max of the row (log2 units) that P and l are expressed
     // against.  It only moves when a tile's max exceeds it by more than
     // kRescaleThreshold, so P <= 2^threshold and O is rescaled rarely; the
@@ -257,7 +261,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < BN; ++c) {
           float x = __uint_as_float(sr[c]) * p.scale_log2;
-          if constexpr (HAS_BIAS) x = fmaf(__ldg(brow + min(kbase + c, len_k - 1)), kLog2e, x);
+          if constexpr (BIAS == kBiasDense) x = fmaf(__ldg(brow + min(kbase + c, len_k - 1)), kLog2e, x);
+          if constexpr (BIAS == kBiasAlibi) x = fmaf(neg_slope2, fabsf(static_cast<float>(kbase + c - i - diag)), x);
           sr[c] = __float_as_uint(x);
         }
       }
@@ -368,13 +373,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D, bool HAS_BIAS, bool FAST>
+template <int D, int BIAS, bool FAST>
 int launch_fwd_t(const TcGeom& g, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                  const FwdParams& p, cudaStream_t st) {
   // At least half of the SM's shared memory, so that a second CTA never waits
   // on the 512 TMEM columns this one holds.
   const size_t smem = std::max<size_t>(sizeof(FwdSmem<D>) + 1024, 116 * 1024);
-  auto kern = fwd_sm100_kernel<D, HAS_BIAS, FAST>;
+  auto kern = fwd_sm100_kernel<D, BIAS, FAST>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return ATTN_ERR_CUDA;
   const int max_nq = g.cu_q ? g.max_nq : g.Nq;
@@ -409,6 +414,7 @@ int launch_fwd_sm100(const TcGeom& g, __nv_bfloat16* o, float* lse, cudaStream_t
   p.lse = lse;
   p.bias = g.bias;
   p.bias_bstride = g.bias_bstride;
+  p.alibi = g.alibi;
   p.cu_q = g.cu_q;
   p.cu_k = g.cu_k;
   p.Hq = g.Hq;
@@ -424,13 +430,17 @@ int launch_fwd_sm100(const TcGeom& g, __nv_bfloat16* o, float* lse, cudaStream_t
   p.wait_limit = kWaitLimitCycles;
   if (!p.status) return ATTN_ERR_CUDA;
   // FAST: no bias and a positive scale, so the row max can be taken on raw scores
-  const bool has_bias = g.bias != nullptr, fast = !has_bias && g.scale > 0.f;
+  const bool fast = !g.bias && !g.alibi && g.scale > 0.f;
   if (g.D == 64) {
-    if (has_bias) return launch_fwd_t<64, true, false>(g, mq, mk, mv, p, st);
-    return fast ? launch_fwd_t<64, false, true>(g, mq, mk, mv, p, st) : launch_fwd_t<64, false, false>(g, mq, mk, mv, p, st);
+    if (g.bias) return launch_fwd_t<64, kBiasDense, false>(g, mq, mk, mv, p, st);
+    if (g.alibi) return launch_fwd_t<64, kBiasAlibi, false>(g, mq, mk, mv, p, st);
+    return fast ? launch_fwd_t<64, kBiasNone, true>(g, mq, mk, mv, p, st)
+                : launch_fwd_t<64, kBiasNone, false>(g, mq, mk, mv, p, st);
   }
-  if (has_bias) return launch_fwd_t<128, true, false>(g, mq, mk, mv, p, st);
-  return fast ? launch_fwd_t<128, false, true>(g, mq, mk, mv, p, st) : launch_fwd_t<128, false, false>(g, mq, mk, mv, p, st);
+  if (g.bias) return launch_fwd_t<128, kBiasDense, false>(g, mq, mk, mv, p, st);
+  if (g.alibi) return launch_fwd_t<128, kBiasAlibi, false>(g, mq, mk, mv, p, st);
+  return fast ? launch_fwd_t<128, kBiasNone, true>(g, mq, mk, mv, p, st)
+              : launch_fwd_t<128, kBiasNone, false>(g, mq, mk, mv, p, st);
 }
 
 }  // namespace attn

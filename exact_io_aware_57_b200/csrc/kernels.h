@@ -24,7 +24,7 @@ int* device_status_ptr();
 
 // ----------------------------------------------------------------- fp32 path
 struct F32Params {
-  const float *q, *k, *v, *bias;
+  const float *q, *k, *v, *bias, *alibi;
   float *o, *lse;
   const int *cu_q, *cu_k;   // packed sequences (device) or null
   long long q_bstride, k_bstride, bias_bstride, lse_bstride, lse_hstride;
@@ -51,6 +51,7 @@ struct TcGeom {
   float scale;
   const float* bias;
   long long bias_bstride;
+  const float* alibi;          // per-query-head ALiBi slopes (device) or null
 };
 
 int launch_fwd_sm100(const TcGeom& g, __nv_bfloat16* o, float* lse, cudaStream_t st);

@@ -64,6 +64,7 @@ __global__ void __launch_bounds__(128) fwd_f32_kernel(F32Params p) {
     acc[e] = 0.f;
   }
   const float* brow = p.bias ? p.bias + s.b * p.bias_bstride + ((long long)h * s.nq + i) * s.nk : nullptr;
+  const float slope = p.alibi ? p.alibi[h] : 0.f;
   const int nvis = visible(p, s, i);
   float m = -INFINITY, l = 0.f;
   for (int j = 0; j < nvis; ++j) {
@@ -73,6 +74,7 @@ __global__ void __launch_bounds__(128) fwd_f32_kernel(F32Params p) {
     for (int e = 0; e < E; ++e) dot = fmaf(qv[e], p.k[kv + lane + 32 * e], dot);
     float sc = warp_sum(dot) * p.scale;
     if (brow) sc += brow[j];
+    if (p.alibi) sc -= slope * fabsf(static_cast<float>(j - i - (s.nk - s.nq)));
     const float mn = fmaxf(m, sc);
     if (mn == -INFINITY) continue;
     const float alpha = expf(m - mn);
@@ -133,6 +135,7 @@ __global__ void __launch_bounds__(128) bwd_dq_f32_kernel(F32Params p, const floa
     acc[e] = 0.f;
   }
   const float* brow = p.bias ? p.bias + s.b * p.bias_bstride + ((long long)h * s.nq + i) * s.nk : nullptr;
+  const float slope = p.alibi ? p.alibi[h] : 0.f;
   const int nvis = lse == -INFINITY ? 0 : visible(p, s, i);
   for (int j = 0; j < nvis; ++j) {
     const long long kv = s.b * p.k_bstride + ((long long)(s.k0 + j) * p.Hkv + hk) * D;
@@ -144,6 +147,7 @@ __global__ void __launch_bounds__(128) bwd_dq_f32_kernel(F32Params p, const floa
     }
     float sc = warp_sum(dot) * p.scale;
     if (brow) sc += brow[j];
+    if (p.alibi) sc -= slope * fabsf(static_cast<float>(j - i - (s.nk - s.nq)));
     const float pij = expf(sc - lse);
     const float ds = pij * (warp_sum(dpv) - Di);
 #pragma unroll
@@ -178,6 +182,7 @@ __global__ void __launch_bounds__(128) bwd_dkdv_f32_kernel(F32Params p, const fl
   for (int g = 0; g < G; ++g) {
     const int h = hk * G + g;
     const float* bcol = p.bias ? p.bias + s.b * p.bias_bstride + (long long)h * s.nq * s.nk + j : nullptr;
+    const float slope = p.alibi ? p.alibi[h] : 0.f;
     for (int i = i0; i < s.nq; ++i) {
       const long long li = s.b * p.lse_bstride + (long long)h * p.lse_hstride + s.q0 + i;
       const float lse = p.lse[li];
@@ -191,6 +196,7 @@ __global__ void __launch_bounds__(128) bwd_dkdv_f32_kernel(F32Params p, const fl
       }
       float sc = warp_sum(dot) * p.scale;
       if (bcol) sc += bcol[(long long)i * s.nk];
+      if (p.alibi) sc -= slope * fabsf(static_cast<float>(j - i - (s.nk - s.nq)));
       const float pij = expf(sc - lse);
       const float ds = pij * (warp_sum(dpv) - Drow[li]);
 #pragma unroll

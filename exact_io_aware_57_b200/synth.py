@@ -65,6 +65,19 @@ def alibi_like_bias(h_q: int, n_q: int, n_k: int, rows=None, heads=None,
     return (-0.05 * dist)[None, :, :] * slope[:, None, None]
 
 
+def alibi_like_slopes(h_q: int) -> torch.Tensor:
+    """fp32 slopes (h + 1) * 0.05 / 32 of the grouped workload's bias."""
+    return (torch.arange(h_q, dtype=torch.float32) + 1.0) * (0.05 / 32.0)
+
+
+def bias_from_slopes(slopes, n_q: int, n_k: int) -> torch.Tensor:
+    """Dense fp32 bias B[h, i, j] = -slope_h * |j - (i + n_k - n_q)| (fp32)."""
+    i = torch.arange(n_q)[:, None]
+    j = torch.arange(n_k)[None, :]
+    dist = (j - (i + (n_k - n_q))).abs().to(torch.float32)
+    return -torch.as_tensor(slopes, dtype=torch.float32)[:, None, None] * dist[None]
+
+
 def varlen_lengths(num_seqs: int, lo: int, hi: int, seed: int = 0) -> np.ndarray:
     """Sequence lengths drawn uniformly from [lo, hi] (inclusive)."""
     return np.random.default_rng(int(seed)).integers(lo, hi + 1, size=int(num_seqs))

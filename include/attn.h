@@ -67,6 +67,17 @@ int attn_fwd(const void* q, const void* k, const void* v, const float* bias,
              int n_q, int n_k, int d, float scale, int causal, int dtype, void* stream);
 
 /*
+ * Forward with the additive bias given by per-head ALiBi slopes instead of a
+ * dense tensor: B[h, i, j] = -slope_h * |j - (i + n_k - n_q)|, formed in
+ * registers (the slope-based position bias the grouped-query workload uses,
+ * "Understanding FlashAttention Pt 1", 0.2 Notation: B an additive bias).
+ * alibi_slopes: DEVICE fp32 [h_q] (required).  Otherwise as attn_fwd.
+ */
+int attn_fwd_alibi(const void* q, const void* k, const void* v, const float* alibi_slopes, void* o,
+                   float* lse, int batch, int h_q, int h_kv, int n_q, int n_k, int d, float scale,
+                   int causal, int dtype, void* stream);
+
+/*
  * Bytes of device workspace attn_bwd needs: an fp32 dQ accumulator
  * [batch, n_q, h_q, d] plus the fp32 row terms D_i = dO_i . O_i [batch, h_q, n_q]
  * (each region 256-byte aligned).  Linear in n, never n^2.
@@ -85,6 +96,12 @@ int attn_bwd(const void* q, const void* k, const void* v, const float* bias,
              void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int batch,
              int h_q, int h_kv, int n_q, int n_k, int d, float scale, int causal, int dtype,
              void* stream);
+
+/* Backward of attn_fwd_alibi (same slopes); otherwise as attn_bwd. */
+int attn_bwd_alibi(const void* q, const void* k, const void* v, const float* alibi_slopes,
+                   const void* o, const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                   void* workspace, size_t workspace_bytes, int batch, int h_q, int h_kv, int n_q,
+                   int n_k, int d, float scale, int causal, int dtype, void* stream);
 
 /*
  * attn_bwd without a workspace argument, for callers that cannot allocate

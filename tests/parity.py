@@ -48,14 +48,15 @@ def rel_fro(a, b) -> float:
     return float(np.linalg.norm(a - b) / max(1e-30, np.linalg.norm(b)))
 
 
-def gpu_fwd(inp, causal, scale=None, bias=None):
+def gpu_fwd(inp, causal, scale=None, bias=None, alibi=None):
     from exact_io_aware_57_b200 import attn
 
     q, k, v = (t.cuda() for t in (inp.q, inp.k, inp.v))
     B, Nq, Hq, d = q.shape
     ob, o = guarded_empty((B, Nq, Hq, d), q.dtype)
     lb, lse = guarded_empty((B, Hq, Nq), torch.float32)
-    attn.attn_fwd(q, k, v, bias=None if bias is None else bias.cuda(), causal=causal, scale=scale, out=o, lse=lse)
+    attn.attn_fwd(q, k, v, bias=None if bias is None else bias.cuda(), causal=causal, scale=scale, out=o, lse=lse,
+                  alibi_slopes=None if alibi is None else alibi.cuda())
     torch.cuda.synchronize()
     assert attn.attn_device_status() == 0
     assert guards_intact(ob) and guards_intact(lb), "kernel wrote outside its output"
@@ -106,16 +107,18 @@ def check_fwd_sampled(orc, q, k, v, o, lse, causal, heads, rows, bias_fn=None, s
     return worst_o, worst_l
 
 
-def gpu_fwd_bwd(inp, causal, bias=None, scale=None):
-    """Forward then backward through the C-ABI on cuda:0; returns CPU tensors."""
+def gpu_fwd_bwd(inp, causal, bias=None, scale=None, alibi=None):
+    """Forward then backward through the C-ABI on cuda:0; returns CPU tensors.
+    ``alibi``: fp32 per-head slopes for the in-kernel position bias."""
     from exact_io_aware_57_b200 import attn
 
     q, k, v, do = (t.cuda() for t in (inp.q, inp.k, inp.v, inp.dout))
     bd = None if bias is None else bias.cuda()
-    o, lse = attn.attn_fwd(q, k, v, bias=bd, causal=causal, scale=scale)
+    sd = None if alibi is None else alibi.cuda()
+    o, lse = attn.attn_fwd(q, k, v, bias=bd, causal=causal, scale=scale, alibi_slopes=sd)
     bufs = [guarded_empty(t.shape, t.dtype) for t in (q, k, v)]
     dq, dk, dv = attn.attn_bwd(q, k, v, o, lse, do, bias=bd, causal=causal, scale=scale,
-                               dq=bufs[0][1], dk=bufs[1][1], dv=bufs[2][1])
+                               dq=bufs[0][1], dk=bufs[1][1], dv=bufs[2][1], alibi_slopes=sd)
     torch.cuda.synchronize()
     assert attn.attn_device_status() == 0
     assert all(guards_intact(b[0]) for b in bufs), "backward wrote outside its outputs"
