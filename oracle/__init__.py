@@ -58,6 +58,14 @@ def _f64(a) -> np.ndarray:
     return np.ascontiguousarray(np.asarray(a, dtype=np.float64))
 
 
+def _window(window):
+    """(left, right) window sizes as C ints; None or a negative side is unbounded."""
+    if window is None:
+        return -1, -1
+    wl, wr = window
+    return (-1 if wl is None else int(wl)), (-1 if wr is None else int(wr))
+
+
 class Oracle:
     """ctypes wrapper around one build of ``attn_oracle.c``."""
 
@@ -69,13 +77,13 @@ class Oracle:
         L = self._lib
         i, d, ll = ctypes.c_int, ctypes.c_double, ctypes.c_longlong
         P = _c_dbl_p
-        L.oracle_attn_fwd.argtypes = [P, P, P, P, ll, P, P, i, i, i, i, i, i, d, i]
-        L.oracle_attn_fwd_rows.argtypes = [P, P, P, P, ctypes.POINTER(ll), i, P, P, i, i, i, d, i]
+        L.oracle_attn_fwd.argtypes = [P, P, P, P, ll, P, P, i, i, i, i, i, i, d, i, i, i]
+        L.oracle_attn_fwd_rows.argtypes = [P, P, P, P, ctypes.POINTER(ll), i, P, P, i, i, i, d, i, i, i]
         L.oracle_attn_fwd_varlen.argtypes = [P, P, P, ctypes.POINTER(ctypes.c_int),
-                                             ctypes.POINTER(ctypes.c_int), i, P, P, i, i, i, d, i]
-        L.oracle_attn_fwd_stream.argtypes = [P, P, P, P, ll, P, P, i, i, i, i, i, i, d, i, i,
+                                             ctypes.POINTER(ctypes.c_int), i, P, P, i, i, i, d, i, i, i]
+        L.oracle_attn_fwd_stream.argtypes = [P, P, P, P, ll, P, P, i, i, i, i, i, i, d, i, i, i, i,
                                              ctypes.POINTER(ll)]
-        L.oracle_attn_bwd.argtypes = [P, P, P, P, ll, P, P, P, P, i, i, i, i, i, i, d, i]
+        L.oracle_attn_bwd.argtypes = [P, P, P, P, ll, P, P, P, P, i, i, i, i, i, i, d, i, i, i]
         L.oracle_merge_partials.argtypes = [P, P, i, i, i, P, P]
         for f in (L.oracle_attn_fwd, L.oracle_attn_fwd_rows, L.oracle_attn_fwd_varlen,
                   L.oracle_attn_fwd_stream, L.oracle_attn_bwd, L.oracle_merge_partials):
@@ -93,9 +101,11 @@ class Oracle:
         assert b.size % per == 0, "bias must be [Hq,Nq,Nk] or [B,Hq,Nq,Nk]"
         return b, per
 
-    def fwd(self, q, k, v, bias=None, causal=False, scale=None):
+    def fwd(self, q, k, v, bias=None, causal=False, scale=None, window=None):
         """O, LSE of softmax(scale*QK^T + B)V.  q [B,Nq,Hq,d], k/v [B,Nk,Hkv,d];
-        returns o [B,Nq,Hq,d] and lse [B,Hq,Nq] (fp64)."""
+        returns o [B,Nq,Hq,d] and lse [B,Hq,Nq] (fp64).  window = (left, right):
+        with a = i + Nk - Nq, keys a - left .. a + right are visible (negative:
+        unbounded on that side)."""
         q, k, v = _f64(q), _f64(k), _f64(v)
         B, Nq, Hq, d = q.shape
         Nk, Hkv = k.shape[1], k.shape[2]
@@ -105,10 +115,10 @@ class Oracle:
         lse = np.zeros((B, Hq, Nq))
         self._lib.oracle_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(b) if b is not None else None,
                                   bstride, _ptr(o), _ptr(lse), B, Hq, Hkv, Nq, Nk, d, scale,
-                                  int(bool(causal)))
+                                  int(bool(causal)), *_window(window))
         return o, lse
 
-    def fwd_stream(self, q, k, v, bias=None, causal=False, scale=None, block=128):
+    def fwd_stream(self, q, k, v, bias=None, causal=False, scale=None, block=128, window=None):
         """Streaming (m, l, a) replay with key blocks of ``block``; returns o, lse, rescales."""
         q, k, v = _f64(q), _f64(k), _f64(v)
         B, Nq, Hq, d = q.shape
@@ -120,10 +130,10 @@ class Oracle:
         cnt = ctypes.c_longlong(0)
         self._lib.oracle_attn_fwd_stream(_ptr(q), _ptr(k), _ptr(v), _ptr(b) if b is not None else None,
                                          bstride, _ptr(o), _ptr(lse), B, Hq, Hkv, Nq, Nk, d, scale,
-                                         int(bool(causal)), int(block), ctypes.byref(cnt))
+                                         int(bool(causal)), *_window(window), int(block), ctypes.byref(cnt))
         return o, lse, cnt.value
 
-    def fwd_rows(self, q_rows, k_head, v_head, rows, Nq, bias_rows=None, causal=False, scale=None):
+    def fwd_rows(self, q_rows, k_head, v_head, rows, Nq, bias_rows=None, causal=False, scale=None, window=None):
         """Forward of selected rows of one (batch, head).  q_rows [R,d], k/v_head [Nk,d],
         rows: query indices of q_rows; bias_rows [R,Nk] or None."""
         q_rows, k_head, v_head = _f64(q_rows), _f64(k_head), _f64(v_head)
@@ -137,10 +147,11 @@ class Oracle:
         self._lib.oracle_attn_fwd_rows(_ptr(q_rows), _ptr(k_head), _ptr(v_head),
                                        _ptr(br) if br is not None else None,
                                        rows.ctypes.data_as(ctypes.POINTER(ctypes.c_longlong)), R,
-                                       _ptr(o), _ptr(lse), int(Nq), Nk, d, scale, int(bool(causal)))
+                                       _ptr(o), _ptr(lse), int(Nq), Nk, d, scale, int(bool(causal)),
+                                       *_window(window))
         return o, lse
 
-    def fwd_varlen(self, q, k, v, cu_q, cu_k, causal=False, scale=None):
+    def fwd_varlen(self, q, k, v, cu_q, cu_k, causal=False, scale=None, window=None):
         """Packed forward.  q [Tq,Hq,d], k/v [Tk,Hkv,d]; returns o [Tq,Hq,d], lse [Hq,Tq]."""
         q, k, v = _f64(q), _f64(k), _f64(v)
         Tq, Hq, d = q.shape
@@ -153,11 +164,11 @@ class Oracle:
         ip = ctypes.POINTER(ctypes.c_int)
         self._lib.oracle_attn_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), cq.ctypes.data_as(ip),
                                          ck.ctypes.data_as(ip), len(cq) - 1, _ptr(o), _ptr(lse),
-                                         Hq, Hkv, d, scale, int(bool(causal)))
+                                         Hq, Hkv, d, scale, int(bool(causal)), *_window(window))
         return o, lse
 
     # ----------------------------------------------------------------- backward
-    def bwd(self, q, k, v, dout, bias=None, causal=False, scale=None):
+    def bwd(self, q, k, v, dout, bias=None, causal=False, scale=None, window=None):
         """dQ, dK, dV of the forward above for upstream gradient dout (fp64)."""
         q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
         B, Nq, Hq, d = q.shape
@@ -169,7 +180,7 @@ class Oracle:
         dv = np.zeros_like(v)
         self._lib.oracle_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(b) if b is not None else None,
                                   bstride, _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
-                                  B, Hq, Hkv, Nq, Nk, d, scale, int(bool(causal)))
+                                  B, Hq, Hkv, Nq, Nk, d, scale, int(bool(causal)), *_window(window))
         return dq, dk, dv
 
     # -------------------------------------------------------------------- merge

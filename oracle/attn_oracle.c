@@ -24,6 +24,10 @@
  * Readings where the pages are silent:
  *   causal: key j is visible from query i iff j <= i + (Nk - Nq) (bottom-right
  *           alignment, so j <= i when Nq == Nk);
+ *   local (sliding-window) attention ("Understanding FlashAttention Pt 1",
+ *           contents 4.2, title only): with a = i + (Nk - Nq), key j is visible
+ *           iff a - window_left <= j <= a + window_right; a negative window is
+ *           unbounded on that side, and causal caps the right side at 0;
  *   a row with no visible key (or every score -inf) has o = 0, LSE = -inf and
  *           zero gradients;
  *   GQA: query head h reads KV head h / (Hq / Hkv).
@@ -48,16 +52,34 @@ static inline long long idx4(long long b, long long n, long long h, long long c,
   return ((b * N + n) * H + h) * D + c;
 }
 
-/* Number of keys visible from query row i (keys 0 .. count-1). */
-static inline long long visible_keys(long long i, long long Nq, long long Nk, int causal) {
-  if (!causal) return Nk;
+/* Keys *lo .. *lo + count - 1 are visible from query row i; returns count. */
+static inline long long key_range(long long i, long long Nq, long long Nk, int causal,
+                                  int wl, int wr, long long* lo) {
+  const long long a = i + (Nk - Nq); /* the key aligned with row i */
+  long long first = 0, end = Nk;
+  if (causal) {
 #if ORACLE_MUTANT == 3
-  long long last = i + (Nk - Nq) - 1; /* planted: off-by-one diagonal */
+    const long long last = a - 1; /* planted: off-by-one diagonal */
 #else
-  long long last = i + (Nk - Nq);
+    const long long last = a;
 #endif
-  if (last < 0) return 0;
-  return last + 1 < Nk ? last + 1 : Nk;
+    if (last + 1 < end) end = last + 1;
+  }
+  if (wr >= 0 && a + wr + 1 < end) end = a + wr + 1;
+#if ORACLE_MUTANT == 11
+  if (wl >= 0 && a - wl + 1 > first) first = a - wl + 1; /* planted: window one key short */
+#else
+  if (wl >= 0 && a - wl > first) first = a - wl;
+#endif
+  *lo = first;
+  return end > first ? end - first : 0;
+}
+
+/* The same range as [*lo, end): returns end. */
+static inline long long lo_end(long long i, long long Nq, long long Nk, int causal, int wl, int wr,
+                               long long* lo) {
+  const long long n = key_range(i, Nq, Nk, causal, wl, wr, lo);
+  return *lo + n;
 }
 
 static inline int kv_head_of(int h, int Hq, int Hkv) {
@@ -130,7 +152,7 @@ static void fwd_row(const double* qi, const double* kbase, const double* vbase,
 void oracle_attn_fwd(const double* q, const double* k, const double* v,
                      const double* bias, long long bias_bstride,
                      double* o, double* lse, int B, int Hq, int Hkv, int Nq, int Nk,
-                     int d, double scale, int causal) {
+                     int d, double scale, int causal, int wl, int wr) {
   const long long nbh = (long long)B * Hq;
 #pragma omp parallel
   {
@@ -143,9 +165,11 @@ void oracle_attn_fwd(const double* q, const double* k, const double* v,
       const double* vb = v + idx4(b, 0, hk, 0, Nk, Hkv, d);
       for (long long i = 0; i < Nq; ++i) {
         const double* brow = bias ? bias + b * bias_bstride + ((long long)h * Nq + i) * Nk : NULL;
-        fwd_row(q + idx4(b, i, h, 0, Nq, Hq, d), kb, vb, (long long)Hkv * d, brow,
-                visible_keys(i, Nq, Nk, causal), d, scale, s, NULL,
-                o + idx4(b, i, h, 0, Nq, Hq, d), lse + ((long long)b * Hq + h) * Nq + i);
+        long long lo;
+        const long long nvis = key_range(i, Nq, Nk, causal, wl, wr, &lo);
+        const long long kvs = (long long)Hkv * d;
+        fwd_row(q + idx4(b, i, h, 0, Nq, Hq, d), kb + lo * kvs, vb + lo * kvs, kvs, brow ? brow + lo : NULL,
+                nvis, d, scale, s, NULL, o + idx4(b, i, h, 0, Nq, Hq, d), lse + ((long long)b * Hq + h) * Nq + i);
       }
     }
     free(s);
@@ -161,15 +185,16 @@ void oracle_attn_fwd(const double* q, const double* k, const double* v,
 void oracle_attn_fwd_rows(const double* q_rows, const double* k_head, const double* v_head,
                           const double* bias_rows, const long long* rows, int R,
                           double* o_rows, double* lse_rows, int Nq, int Nk, int d,
-                          double scale, int causal) {
+                          double scale, int causal, int wl, int wr) {
 #pragma omp parallel
   {
     double* s = (double*)malloc(sizeof(double) * (Nk > 0 ? Nk : 1));
 #pragma omp for schedule(dynamic, 1)
     for (int r = 0; r < R; ++r) {
-      fwd_row(q_rows + (long long)r * d, k_head, v_head, d,
-              bias_rows ? bias_rows + (long long)r * Nk : NULL,
-              visible_keys(rows[r], Nq, Nk, causal), d, scale, s, NULL,
+      long long lo;
+      const long long nvis = key_range(rows[r], Nq, Nk, causal, wl, wr, &lo);
+      fwd_row(q_rows + (long long)r * d, k_head + lo * d, v_head + lo * d, d,
+              bias_rows ? bias_rows + (long long)r * Nk + lo : NULL, nvis, d, scale, s, NULL,
               o_rows + (long long)r * d, lse_rows + r);
     }
     free(s);
@@ -182,7 +207,7 @@ void oracle_attn_fwd_rows(const double* q_rows, const double* k_head, const doub
 void oracle_attn_fwd_varlen(const double* q, const double* k, const double* v,
                             const int* cu_q, const int* cu_k, int nseq,
                             double* o, double* lse, int Hq, int Hkv, int d,
-                            double scale, int causal) {
+                            double scale, int causal, int wl, int wr) {
   const long long Tq = cu_q[nseq];
   int maxk = 1;
   for (int z = 0; z < nseq; ++z) if (cu_k[z + 1] - cu_k[z] > maxk) maxk = cu_k[z + 1] - cu_k[z];
@@ -199,9 +224,11 @@ void oracle_attn_fwd_varlen(const double* q, const double* k, const double* v,
       const double* kb = k + (k0 * Hkv + hk) * d;
       const double* vb = v + (k0 * Hkv + hk) * d;
       for (long long i = 0; i < nq; ++i) {
-        fwd_row(q + ((q0 + i) * Hq + h) * d, kb, vb, (long long)Hkv * d, NULL,
-                visible_keys(i, nq, nk, causal), d, scale, s, NULL,
-                o + ((q0 + i) * Hq + h) * d, lse + (long long)h * Tq + q0 + i);
+        long long lo;
+        const long long nvis = key_range(i, nq, nk, causal, wl, wr, &lo);
+        const long long kvs = (long long)Hkv * d;
+        fwd_row(q + ((q0 + i) * Hq + h) * d, kb + lo * kvs, vb + lo * kvs, kvs, NULL, nvis, d, scale, s,
+                NULL, o + ((q0 + i) * Hq + h) * d, lse + (long long)h * Tq + q0 + i);
       }
     }
     free(s);
@@ -219,7 +246,8 @@ void oracle_attn_fwd_varlen(const double* q, const double* k, const double* v,
 void oracle_attn_fwd_stream(const double* q, const double* k, const double* v,
                             const double* bias, long long bias_bstride,
                             double* o, double* lse, int B, int Hq, int Hkv, int Nq, int Nk,
-                            int d, double scale, int causal, int block, long long* rescales) {
+                            int d, double scale, int causal, int wl, int wr, int block,
+                            long long* rescales) {
   const long long nbh = (long long)B * Hq;
   long long total = 0;
 #pragma omp parallel reduction(+ : total)
@@ -233,11 +261,12 @@ void oracle_attn_fwd_stream(const double* q, const double* k, const double* v,
       for (long long i = 0; i < Nq; ++i) {
         const double* qi = q + idx4(b, i, h, 0, Nq, Hq, d);
         const double* brow = bias ? bias + b * bias_bstride + ((long long)h * Nq + i) * Nk : NULL;
-        const long long nvis = visible_keys(i, Nq, Nk, causal);
+        long long lo;
+        const long long end = lo_end(i, Nq, Nk, causal, wl, wr, &lo);
         double m = -INFINITY, l = 0.0;
         for (int c = 0; c < d; ++c) a[c] = 0.0;
-        for (long long j0 = 0; j0 < nvis; j0 += block) {
-          const long long nb = nvis - j0 < block ? nvis - j0 : block;
+        for (long long j0 = lo; j0 < end; j0 += block) {
+          const long long nb = end - j0 < block ? end - j0 : block;
           const double mb = row_scores(qi, k + idx4(b, j0, hk, 0, Nk, Hkv, d), (long long)Hkv * d,
                                        brow ? brow + j0 : NULL, nb, d, scale, sb);
           const double mnew = mb > m ? mb : m;
@@ -283,7 +312,7 @@ void oracle_attn_fwd_stream(const double* q, const double* k, const double* v,
 void oracle_attn_bwd(const double* q, const double* k, const double* v,
                      const double* bias, long long bias_bstride, const double* dout,
                      double* dq, double* dk, double* dv, int B, int Hq, int Hkv, int Nq,
-                     int Nk, int d, double scale, int causal) {
+                     int Nk, int d, double scale, int causal, int wl, int wr) {
   const int G = Hq / Hkv;
   const long long nbk = (long long)B * Hkv;
   memset(dk, 0, sizeof(double) * (size_t)B * Nk * Hkv * d);
@@ -308,18 +337,21 @@ void oracle_attn_bwd(const double* q, const double* k, const double* v,
           const double* doi = dout + idx4(b, i, h, 0, Nq, Hq, d);
           double* dqi = dq + idx4(b, i, h, 0, Nq, Hq, d);
           const double* brow = bias ? bias + b * bias_bstride + ((long long)h * Nq + i) * Nk : NULL;
-          const long long nvis = visible_keys(i, Nq, Nk, causal);
+          long long lo;
+          const long long nvis = key_range(i, Nq, Nk, causal, wl, wr, &lo);
+          const long long kvs = (long long)Hkv * d;
           double lse_i;
-          fwd_row(qi, kb, vb, (long long)Hkv * d, brow, nvis, d, scale, s, p, oi, &lse_i);
+          fwd_row(qi, kb + lo * kvs, vb + lo * kvs, kvs, brow ? brow + lo : NULL, nvis, d, scale, s, p, oi,
+                  &lse_i);
           for (int c = 0; c < d; ++c) dqi[c] = 0.0;
           if (lse_i == -INFINITY) continue;
           double Di = 0.0;
           for (int c = 0; c < d; ++c) Di += doi[c] * oi[c];
-          for (long long j = 0; j < nvis; ++j) {
-            const double* kj = kb + j * (long long)Hkv * d;
-            const double* vj = vb + j * (long long)Hkv * d;
-            double* dkj = dk + idx4(b, j, hk, 0, Nk, Hkv, d);
-            double* dvj = dv + idx4(b, j, hk, 0, Nk, Hkv, d);
+          for (long long j = 0; j < nvis; ++j) { /* key lo + j; p[j] is its probability */
+            const double* kj = kb + (lo + j) * kvs;
+            const double* vj = vb + (lo + j) * kvs;
+            double* dkj = dk + idx4(b, lo + j, hk, 0, Nk, Hkv, d);
+            double* dvj = dv + idx4(b, lo + j, hk, 0, Nk, Hkv, d);
             double dP = 0.0;
             for (int c = 0; c < d; ++c) dP += doi[c] * vj[c];
 #if ORACLE_MUTANT == 6

@@ -12,7 +12,10 @@ Sources:
     handbook's 0.2 Notation);
   * library special case: scipy's logsumexp/softmax on the plain
     non-causal problem;
-  * backward: central finite differences of the forward in fp64.
+  * backward: central finite differences of the forward in fp64;
+  * local (sliding-window) attention, named in the handbook's contents (4.2)
+    without a definition: the reading a - left <= j <= a + right with
+    a = i + Nk - Nq is checked against scipy's softmax over exactly that slice.
 """
 from __future__ import annotations
 
@@ -176,8 +179,8 @@ def pin_library_softmax(orc):
     return worst <= 1e-13, f"max rel err {worst:.2e}"
 
 
-def _loss(orc, q, k, v, dout, bias, causal):
-    o, _ = orc.fwd(q, k, v, bias=bias, causal=causal)
+def _loss(orc, q, k, v, dout, bias, causal, window=None):
+    o, _ = orc.fwd(q, k, v, bias=bias, causal=causal, window=window)
     return float(np.sum(o * dout))
 
 
@@ -185,15 +188,17 @@ def pin_backward_fd(orc):
     """Central finite differences (step 1e-6) of sum(dO * O) w.r.t. Q, K, V."""
     rng = np.random.default_rng(19)
     worst = 0.0
-    for (B, nq, nk, hq, hkv, d, causal, use_bias) in ((1, 5, 5, 2, 1, 4, True, True),
-                                                       (1, 3, 6, 2, 2, 3, False, False),
-                                                       (2, 4, 4, 1, 1, 2, True, False)):
+    for (B, nq, nk, hq, hkv, d, causal, use_bias, window) in ((1, 5, 5, 2, 1, 4, True, True, None),
+                                                               (1, 3, 6, 2, 2, 3, False, False, None),
+                                                               (2, 4, 4, 1, 1, 2, True, False, None),
+                                                               (1, 6, 6, 2, 1, 3, True, True, (2, -1)),
+                                                               (1, 5, 7, 1, 1, 2, False, False, (1, 1))):
         q = _rand(rng, B, nq, hq, d)
         k = _rand(rng, B, nk, hkv, d)
         v = _rand(rng, B, nk, hkv, d)
         dout = _rand(rng, B, nq, hq, d)
         bias = _rand(rng, hq, nq, nk) if use_bias else None
-        dq, dk, dv = orc.bwd(q, k, v, dout, bias=bias, causal=causal)
+        dq, dk, dv = orc.bwd(q, k, v, dout, bias=bias, causal=causal, window=window)
         for x, g in ((q, dq), (k, dk), (v, dv)):
             num = np.zeros_like(x)
             it = np.nditer(x, flags=["multi_index"])
@@ -201,9 +206,9 @@ def pin_backward_fd(orc):
                 idx = it.multi_index
                 old = x[idx]
                 x[idx] = old + 1e-6
-                lp = _loss(orc, q, k, v, dout, bias, causal)
+                lp = _loss(orc, q, k, v, dout, bias, causal, window)
                 x[idx] = old - 1e-6
-                lm = _loss(orc, q, k, v, dout, bias, causal)
+                lm = _loss(orc, q, k, v, dout, bias, causal, window)
                 x[idx] = old
                 num[idx] = (lp - lm) / 2e-6
             worst = max(worst, float(np.linalg.norm(g - num) / max(1e-300, np.linalg.norm(num))))
@@ -228,7 +233,43 @@ def pin_gqa_sum(orc):
     return worst <= 1e-12, f"max rel err {worst:.2e}"
 
 
+def pin_window_slices(orc):
+    """Local attention: row i equals scipy's softmax over exactly the keys
+    a - left .. a + right (a = i + Nk - Nq; causal caps the right side at a;
+    a negative size is unbounded), and with left = 0 under causal the single
+    key a is left, so o_i = v_a."""
+    rng = np.random.default_rng(21)
+    worst = 0.0
+    d = 4
+    for (nq, nk, wl, wr, causal) in ((9, 9, 2, -1, True), (9, 9, 0, -1, True), (7, 11, 3, 1, False),
+                                     (11, 7, 1, 2, False), (8, 8, -1, 2, False), (6, 10, 4, 5, True),
+                                     (10, 4, 1, -1, True)):
+        q = _rand(rng, 1, nq, 2, d, scale=1.5)
+        k = _rand(rng, 1, nk, 1, d, scale=1.5)
+        v = _rand(rng, 1, nk, 1, d)
+        bias = _rand(rng, 2, nq, nk)
+        o, l = orc.fwd(q, k, v, bias=bias, causal=causal, window=(wl, wr))
+        for h in range(2):
+            for i in range(nq):
+                a = i + nk - nq
+                lo = 0 if wl < 0 else max(0, a - wl)
+                hi = nk - 1 if wr < 0 else min(nk - 1, a + wr)
+                if causal:
+                    hi = min(hi, a)
+                if hi < lo:
+                    if not (np.all(o[0, i, h] == 0.0) and l[0, h, i] == -np.inf):
+                        return False, f"row {i} has no visible key but o/LSE are not 0/-inf"
+                    continue
+                s = q[0, i, h] @ k[0, lo:hi + 1, 0].T / math.sqrt(d) + bias[h, i, lo:hi + 1]
+                worst = max(worst, float(np.max(np.abs(o[0, i, h] - softmax(s) @ v[0, lo:hi + 1, 0]))),
+                            abs(float(l[0, h, i] - logsumexp(s))))
+        if causal and wl == 0 and nq == nk:
+            worst = max(worst, float(np.max(np.abs(o[0, :, :, :] - v[0, :, 0, None, :]))))
+    return worst <= 1e-13, f"max abs err {worst:.2e}"
+
+
 ALL_PINS = {
+    "window_slices": pin_window_slices,
     "merge_every_split": pin_merge_every_split,
     "stream_equals_oneshot": pin_stream_equals_oneshot,
     "constant_scores": pin_constant_scores,

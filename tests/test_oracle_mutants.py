@@ -16,6 +16,7 @@ MUTANTS = {
     8: "dS used in place of P for dV",
     9: "running state not rescaled when the max grows",
     10: "K used in place of V in the output",
+    11: "local window one key short on the left",
 }
 
 
