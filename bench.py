@@ -56,6 +56,8 @@ def parse_args(argv=None):
     ap.add_argument("--heads", type=int, default=None, help="override the head count (profiling a smaller case)")
     ap.add_argument("--bias-mode", default="dense", choices=["dense", "alibi"],
                     help="grouped workload: read the dense fp32 bias tensor, or form it in-kernel from slopes")
+    ap.add_argument("--window", type=int, default=None,
+                    help="causal sliding window: each row sees its own and at most WINDOW earlier keys")
     ap.add_argument("--naive", action="store_true",
                     help="time the fused forward against the materialising three-kernel comparator instead")
     return ap.parse_args(argv)
@@ -269,6 +271,7 @@ def make_job(w, args, dev, rank):
             j.host["alibi"] = synth.alibi_like_slopes(w.h_q).pin_memory()
         j.dev = {n: t.to(dev) for n, t in j.host.items()}
         j.out = {"o": torch.empty_like(j.dev["q"]), "lse": torch.empty((w.batch, w.h_q, w.n), device=dev)}
+        win = None if args.window is None else (int(args.window), None)
         ws = None
         if w.backward:
             j.out.update(dq=torch.empty_like(j.dev["q"]), dk=torch.empty_like(j.dev["k"]),
@@ -278,11 +281,11 @@ def make_job(w, args, dev, rank):
         def step():
             d_, o_ = j.dev, j.out
             attn.attn_fwd(d_["q"], d_["k"], d_["v"], bias=d_.get("bias"), causal=w.causal, out=o_["o"], lse=o_["lse"],
-                          alibi_slopes=d_.get("alibi"))
+                          alibi_slopes=d_.get("alibi"), window=win)
             if w.backward:
                 attn.attn_bwd(d_["q"], d_["k"], d_["v"], o_["o"], o_["lse"], d_["dout"], bias=d_.get("bias"),
                               causal=w.causal, workspace=ws, dq=o_["dq"], dk=o_["dk"], dv=o_["dv"],
-                              alibi_slopes=d_.get("alibi"))
+                              alibi_slopes=d_.get("alibi"), window=win)
     j.step = step
     j.out_host = {n: torch.empty(t.shape, dtype=t.dtype).pin_memory() for n, t in j.out.items()}
 
@@ -363,8 +366,8 @@ def run_ours(args):
         fwd_ms = max_over_ranks(dist, statistics.mean(a.elapsed_time(b) for a, b in fwd_ev), dev)
         if w.backward:
             bwd_main_ms = max_over_ranks(dist, statistics.mean(a.elapsed_time(b) for a, b in bwd_ev), dev)
-    f_fwd = workloads.flops(w, backward=False, lengths=job.lengths)
-    f_step = workloads.flops(w, lengths=job.lengths)
+    f_fwd = workloads.flops(w, backward=False, lengths=job.lengths, window=args.window)
+    f_step = workloads.flops(w, lengths=job.lengths, window=args.window)
     value = world * f_step / (ms_step * 1e-3) / 1e12
 
     # ---- end to end through the public API with pinned host buffers
@@ -425,6 +428,7 @@ def run_ours(args):
                        "head_dim": w.d, "causal": w.causal,
                        "bias": (("dense fp32 tensor" if args.bias_mode == "dense" else "per-head slopes, formed in-kernel")
                                 if w.bias else False), "backward": w.backward,
+                       "window": None if args.window is None else f"causal, keys i-{args.window}..i",
                        "global_batch": w.batch * world, "parallelism": f"dp{world} (independent problem per GPU)",
                        "l2": l2_note},
             "fwd_tflops": round(world * f_fwd / (fwd_ms * 1e-3) / 1e12, 2) if fwd_ms else None,

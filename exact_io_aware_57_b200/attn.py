@@ -35,6 +35,9 @@ EXPORTS = {
     "attn_fwd_alibi": (_I, [_VP, _VP, _VP, _FP, _VP, _FP, _I, _I, _I, _I, _I, _I, _F, _I, _I, _VP]),
     "attn_bwd_alibi": (_I, [_VP, _VP, _VP, _FP, _VP, _FP, _VP, _VP, _VP, _VP, _VP, _SZ, _I, _I, _I, _I, _I, _I,
                             _F, _I, _I, _VP]),
+    "attn_fwd_local": (_I, [_VP, _VP, _VP, _FP, _VP, _FP, _I, _I, _I, _I, _I, _I, _F, _I, _I, _I, _I, _VP]),
+    "attn_bwd_local": (_I, [_VP, _VP, _VP, _FP, _VP, _FP, _VP, _VP, _VP, _VP, _VP, _SZ, _I, _I, _I, _I, _I, _I,
+                            _F, _I, _I, _I, _I, _VP]),
     "attn_bwd_workspace_size": (_SZ, [_I, _I, _I, _I]),
     "attn_bwd": (_I, [_VP, _VP, _VP, _FP, _LL, _VP, _FP, _VP, _VP, _VP, _VP, _VP, _SZ, _I, _I, _I, _I, _I,
                       _I, _F, _I, _I, _VP]),
@@ -121,15 +124,32 @@ def _slopes(alibi_slopes, Hq):
     return _dev(alibi_slopes, "alibi_slopes")
 
 
-def attn_fwd(q, k, v, bias=None, causal=False, scale=None, out=None, lse=None, stream=None, alibi_slopes=None):
+def _window_args(window, bias):
+    if bias is not None:
+        raise AttnError("a local window takes alibi_slopes, not a dense bias")
+    wl, wr = window
+    return (-1 if wl is None else int(wl)), (-1 if wr is None else int(wr))
+
+
+def attn_fwd(q, k, v, bias=None, causal=False, scale=None, out=None, lse=None, stream=None, alibi_slopes=None,
+             window=None):
     """O, LSE = attention(q [B,Nq,Hq,d], k/v [B,Nk,Hkv,d]); o like q, lse fp32 [B,Hq,Nq].
     bias: dense fp32 [Hq,Nq,Nk] or [B,Hq,Nq,Nk]; alibi_slopes: fp32 [Hq] (bias
-    -slope_h |j - (i + Nk - Nq)| formed in the kernel); at most one of the two."""
+    -slope_h |j - (i + Nk - Nq)| formed in the kernel); at most one of the two.
+    window = (left, right): local attention, keys a - left .. a + right of the
+    key a = i + Nk - Nq aligned with row i (None or negative: unbounded)."""
     B, Nq, Hq, d = q.shape
     Nk, Hkv = k.shape[1], k.shape[2]
     scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
     o = torch.empty_like(q) if out is None else out
     lse = torch.empty((B, Hq, Nq), device=q.device, dtype=torch.float32) if lse is None else lse
+    if window is not None:
+        wl, wr = _window_args(window, bias)
+        _check(_lib.attn_fwd_local(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"),
+                                   None if alibi_slopes is None else _slopes(alibi_slopes, Hq), _dev(o, "o"),
+                                   _dev(lse, "lse"), B, Hq, Hkv, Nq, Nk, d, scale, int(bool(causal)), wl, wr,
+                                   _dtype_code(q), _stream(stream)))
+        return o, lse
     if alibi_slopes is not None:
         if bias is not None:
             raise AttnError("pass either bias or alibi_slopes")
@@ -148,7 +168,7 @@ def attn_bwd_workspace_size(batch, h_q, n_q, d) -> int:
 
 
 def attn_bwd(q, k, v, o, lse, dout, bias=None, causal=False, scale=None, workspace=None, dq=None, dk=None,
-             dv=None, stream=None, alibi_slopes=None):
+             dv=None, stream=None, alibi_slopes=None, window=None):
     """dq, dk, dv of attn_fwd for upstream gradient dout (layouts as q, k, v)."""
     B, Nq, Hq, d = q.shape
     Nk, Hkv = k.shape[1], k.shape[2]
@@ -159,6 +179,15 @@ def attn_bwd(q, k, v, o, lse, dout, bias=None, causal=False, scale=None, workspa
     need = attn_bwd_workspace_size(B, Hq, Nq, d)
     if workspace is None:
         workspace = torch.empty(need, device=q.device, dtype=torch.uint8)
+    if window is not None:
+        wl, wr = _window_args(window, bias)
+        _check(_lib.attn_bwd_local(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"),
+                                   None if alibi_slopes is None else _slopes(alibi_slopes, Hq), _dev(o, "o"),
+                                   _dev(lse, "lse"), _dev(dout, "dout"), _dev(dq, "dq"), _dev(dk, "dk"),
+                                   _dev(dv, "dv"), _dev(workspace, "workspace"),
+                                   workspace.numel() * workspace.element_size(), B, Hq, Hkv, Nq, Nk, d, scale,
+                                   int(bool(causal)), wl, wr, _dtype_code(q), _stream(stream)))
+        return dq, dk, dv
     if alibi_slopes is not None:
         if bias is not None:
             raise AttnError("pass either bias or alibi_slopes")

@@ -101,20 +101,13 @@ int check_common(int batch, int h_q, int h_kv, int n_q, int n_k, int d, int dtyp
   if (dtype != ATTN_BF16 && dtype != ATTN_F32) return ATTN_ERR_UNSUPPORTED;
   // the kernels index rows with 32-bit coordinates (TMA) and 64-bit offsets
   if ((long long)batch * n_q > (1ll << 31) - 1 || (long long)batch * n_k > (1ll << 31) - 1) return ATTN_ERR_INVALID;
+  if (n_q > kMaxSeqLen || n_k > kMaxSeqLen) return ATTN_ERR_UNSUPPORTED;
   return ATTN_OK;
 }
 
-}  // namespace
-
-extern "C" {
-
-}  // extern "C"
-
-namespace {
-
 int fwd_impl(const void* q, const void* k, const void* v, const float* bias, long long bias_batch_stride,
              const float* alibi, void* o, float* lse, int batch, int h_q, int h_kv, int n_q, int n_k, int d,
-             float scale, int causal, int dtype, void* stream) {
+             float scale, int causal, int window_left, int window_right, int dtype, void* stream) {
   int rc = check_common(batch, h_q, h_kv, n_q, n_k, d, dtype);
   if (rc) return rc;
   if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID;
@@ -142,6 +135,8 @@ int fwd_impl(const void* q, const void* k, const void* v, const float* bias, lon
     p.Nk = n_k;
     p.D = d;
     p.causal = causal != 0;
+    p.window_left = window_left;
+    p.window_right = window_right;
     p.scale = scale;
     return launch_fwd_f32(p, batch, n_q, st);
   }
@@ -156,6 +151,8 @@ int fwd_impl(const void* q, const void* k, const void* v, const float* bias, lon
   g.Nk = n_k;
   g.D = d;
   g.causal = causal != 0;
+  g.window_left = window_left;
+  g.window_right = window_right;
   g.scale = scale;
   g.bias = bias;
   g.bias_bstride = bias_batch_stride;
@@ -171,15 +168,22 @@ int attn_fwd(const void* q, const void* k, const void* v, const float* bias, lon
              float* lse, int batch, int h_q, int h_kv, int n_q, int n_k, int d, float scale, int causal, int dtype,
              void* stream) {
   return fwd_impl(q, k, v, bias, bias_batch_stride, nullptr, o, lse, batch, h_q, h_kv, n_q, n_k, d, scale, causal,
-                  dtype, stream);
+                  -1, -1, dtype, stream);
 }
 
 int attn_fwd_alibi(const void* q, const void* k, const void* v, const float* alibi_slopes, void* o, float* lse,
                    int batch, int h_q, int h_kv, int n_q, int n_k, int d, float scale, int causal, int dtype,
                    void* stream) {
   if (!alibi_slopes) return ATTN_ERR_INVALID;
-  return fwd_impl(q, k, v, nullptr, 0, alibi_slopes, o, lse, batch, h_q, h_kv, n_q, n_k, d, scale, causal, dtype,
-                  stream);
+  return fwd_impl(q, k, v, nullptr, 0, alibi_slopes, o, lse, batch, h_q, h_kv, n_q, n_k, d, scale, causal, -1, -1,
+                  dtype, stream);
+}
+
+int attn_fwd_local(const void* q, const void* k, const void* v, const float* alibi_slopes, void* o, float* lse,
+                   int batch, int h_q, int h_kv, int n_q, int n_k, int d, float scale, int causal, int window_left,
+                   int window_right, int dtype, void* stream) {
+  return fwd_impl(q, k, v, nullptr, 0, alibi_slopes, o, lse, batch, h_q, h_kv, n_q, n_k, d, scale, causal,
+                  window_left, window_right, dtype, stream);
 }
 
 size_t attn_bwd_workspace_size(int batch, int h_q, int n_q, int d) {
@@ -194,7 +198,7 @@ namespace {
 int bwd_impl(const void* q, const void* k, const void* v, const float* bias, long long bias_batch_stride,
              const float* alibi, const void* o, const float* lse, const void* dout, void* dq, void* dk, void* dv,
              void* workspace, size_t workspace_bytes, int batch, int h_q, int h_kv, int n_q, int n_k, int d,
-             float scale, int causal, int dtype, void* stream) {
+             float scale, int causal, int window_left, int window_right, int dtype, void* stream) {
   int rc = check_common(batch, h_q, h_kv, n_q, n_k, d, dtype);
   if (rc) return rc;
   if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return ATTN_ERR_INVALID;
@@ -231,6 +235,8 @@ int bwd_impl(const void* q, const void* k, const void* v, const float* bias, lon
     p.Nk = n_k;
     p.D = d;
     p.causal = causal != 0;
+    p.window_left = window_left;
+    p.window_right = window_right;
     p.scale = scale;
     return launch_bwd_f32(p, static_cast<const float*>(dout), Drow, static_cast<float*>(dq), static_cast<float*>(dk),
                           static_cast<float*>(dv), batch, n_q, n_k, st);
@@ -246,6 +252,8 @@ int bwd_impl(const void* q, const void* k, const void* v, const float* bias, lon
   g.Nk = n_k;
   g.D = d;
   g.causal = causal != 0;
+  g.window_left = window_left;
+  g.window_right = window_right;
   g.scale = scale;
   g.bias = bias;
   g.bias_bstride = bias_batch_stride;
@@ -264,7 +272,7 @@ int attn_bwd(const void* q, const void* k, const void* v, const float* bias, lon
              size_t workspace_bytes, int batch, int h_q, int h_kv, int n_q, int n_k, int d, float scale, int causal,
              int dtype, void* stream) {
   return bwd_impl(q, k, v, bias, bias_batch_stride, nullptr, o, lse, dout, dq, dk, dv, workspace, workspace_bytes,
-                  batch, h_q, h_kv, n_q, n_k, d, scale, causal, dtype, stream);
+                  batch, h_q, h_kv, n_q, n_k, d, scale, causal, -1, -1, dtype, stream);
 }
 
 int attn_bwd_alibi(const void* q, const void* k, const void* v, const float* alibi_slopes, const void* o,
@@ -273,7 +281,15 @@ int attn_bwd_alibi(const void* q, const void* k, const void* v, const float* ali
                    int causal, int dtype, void* stream) {
   if (!alibi_slopes) return ATTN_ERR_INVALID;
   return bwd_impl(q, k, v, nullptr, 0, alibi_slopes, o, lse, dout, dq, dk, dv, workspace, workspace_bytes, batch,
-                  h_q, h_kv, n_q, n_k, d, scale, causal, dtype, stream);
+                  h_q, h_kv, n_q, n_k, d, scale, causal, -1, -1, dtype, stream);
+}
+
+int attn_bwd_local(const void* q, const void* k, const void* v, const float* alibi_slopes, const void* o,
+                   const float* lse, const void* dout, void* dq, void* dk, void* dv, void* workspace,
+                   size_t workspace_bytes, int batch, int h_q, int h_kv, int n_q, int n_k, int d, float scale,
+                   int causal, int window_left, int window_right, int dtype, void* stream) {
+  return bwd_impl(q, k, v, nullptr, 0, alibi_slopes, o, lse, dout, dq, dk, dv, workspace, workspace_bytes, batch,
+                  h_q, h_kv, n_q, n_k, d, scale, causal, window_left, window_right, dtype, stream);
 }
 
 int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse, const int* cu_seqlens_q,

@@ -70,6 +70,7 @@ struct BwdParams {
   int Hq, Hkv, Nq, Nk;
   float scale, scale_log2;
   int causal;
+  int win_l, win_r;  // key j visible from query i iff i + diag - win_l <= j <= i + diag + win_r
   int* status;
   long long wait_limit;
 };
@@ -102,13 +103,14 @@ ATTN_DEVINL void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
 // Phase A -- P^T for one key row (this thread) and 128 queries, 32 at a time:
 //   P^T = 2^(scale log2e s + log2e B - log2e LSE), written back into TMEM as
 // bf16 pairs over the S^T columns already read (A operand of dV += P^T dO).
-// MASK zeroes queries this key is hidden from (causal: query i sees key j iff
-// j <= i + diag; padding rows and keys).  Rolled over chunks so the code stays
-// small enough for the instruction cache.
+// MASK zeroes queries this key is hidden from (query i sees key kj iff
+// kj - lo_off <= i <= kj + hi_off, i.e. i + diag - win_l <= kj <= i + diag + win_r;
+// padding rows and keys).  Rolled over chunks so the code stays small enough
+// for the instruction cache.
 template <bool MASK, int BIAS>
 ATTN_DEVINL void bwd_p_chunks(uint32_t st_col, const float* nlse2, float scale_log2, const float* bcol,
-                              float neg_slope2, int nk, int i0, int len_q, int kj, int len_k, int diag,
-                              int bias_diag) {
+                              float neg_slope2, int nk, int i0, int len_q, int kj, int len_k, int lo_off,
+                              int hi_off, int bias_diag) {
 #pragma unroll 1
   for (int c = 0; c < BM / 32; ++c) {
     uint32_t sr[32];
@@ -119,8 +121,8 @@ ATTN_DEVINL void bwd_p_chunks(uint32_t st_col, const float* nlse2, float scale_l
     const int q0 = i0 + c * 32;
     int vis_lo = 0, vis_hi = 32;  // queries q0 + e, vis_lo <= e < vis_hi, see this key
     if constexpr (MASK) {
-      vis_lo = kj - diag - q0;
-      vis_hi = min(32, len_q - q0);
+      vis_lo = kj - lo_off - q0;
+      vis_hi = min(min(32, len_q - q0), kj + hi_off - q0 + 1);
       if (kj >= len_k) vis_hi = 0;
     }
     uint32_t pk[16];
@@ -200,15 +202,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int n_tile = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
   const int n0 = n_tile * BN;
   const int len_q = p.Nq, len_k = p.Nk;
-  const int diag = len_k - len_q;  // key j visible from query i iff j <= i + diag
+  const int diag = len_k - len_q;  // query i is aligned with key i + diag
   const int G = p.Hq / p.Hkv;
-  const int n_qt = (len_q + BM - 1) / BM;
-  int i_first = 0;
-  if (p.causal) {
-    const int first_row = n0 - diag;  // first query row that sees key n0
-    i_first = first_row <= 0 ? 0 : first_row / BM;
-  }
-  const int per_head = i_first < n_qt ? n_qt - i_first : 0;
+  // query rows that see at least one key of n0 .. n0 + BN - 1
+  const int first_row = max(0, n0 - diag - p.win_r);
+  const int last_row = min(len_q - 1, n0 + BN - 1 - diag + p.win_l);
+  const int i_first = first_row / BM;
+  const int per_head = last_row >= first_row ? last_row / BM - i_first + 1 : 0;
   const int n_steps = G * per_head;
 
   if ((smem_u32(smem_raw) & 1023u) != 0) {  // the swizzle needs 1024-byte aligned tiles
@@ -365,7 +365,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_after();
       // tile-level (warp-uniform) condition: the chunk routines hold
       // warp-collective tcgen05 instructions, so every lane must take the same one
-      const bool need_mask = (n0 + BN > len_k) || (i0 + BM > len_q) || (p.causal && n0 + BN - 1 > i0 + diag);
+      const bool need_mask = (n0 + BN > len_k) || (i0 + BM > len_q) || (n0 + BN - 1 > i0 + diag + p.win_r) ||
+                             (n0 < i0 + BM - 1 + diag - p.win_l);
       const float* bcol = nullptr;
       if constexpr (BIAS == kBiasDense) bcol = p.bias + b * p.bias_bstride + (long long)h * p.Nq * p.Nk + min(kj, len_k - 1);
       float neg_slope2 = 0.f;
@@ -373,10 +374,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t st_col = tmem + lane_off + kColST, dp_col = tmem + lane_off + kColDPT;
       if (need_mask)
         bwd_p_chunks<true, BIAS>(st_col, s.nlse2[st], p.scale_log2, bcol, neg_slope2, p.Nk, i0, len_q, kj, len_k,
-                                 p.causal ? diag : (1 << 30), diag);
+                                 diag + p.win_r, p.win_l - diag, diag);
       else
         bwd_p_chunks<false, BIAS>(st_col, s.nlse2[st], p.scale_log2, bcol, neg_slope2, p.Nk, i0, len_q, kj, len_k,
-                                  1 << 30, diag);
+                                  0, 0, diag);
       tmem_wait_st();
       // dS^T needs dP^T, and the shared tile back from the previous dQ drain
       ok = __all_sync(0xffffffffu, mbar_wait(&s.dpt_full, step & 1, ab) &&
@@ -596,6 +597,8 @@ int launch_bwd_sm100(const TcGeom& g, const __nv_bfloat16* o, const float* lse, 
   p.scale = g.scale;
   p.scale_log2 = g.scale * kLog2e;
   p.causal = g.causal;
+  p.win_l = win_left(g.window_left);
+  p.win_r = win_right(g.causal, g.window_right);
   p.status = device_status_ptr();
   p.wait_limit = kWaitLimitCycles;
   if (!p.status) return ATTN_ERR_CUDA;

@@ -23,7 +23,10 @@
 // MMA warp then accumulates O += P V_j.  O / l and LSE = (m + log2 l) ln 2 are
 // written once, after the last tile (the division by l happens a single time,
 // as in the same page's lab).
-// Causal: KV tiles that lie wholly above the diagonal are never loaded.
+// Causal and local (sliding-window) attention: only the KV tiles that hold a
+// key visible from some row of the tile are loaded ("Understanding
+// FlashAttention Pt 1", contents 3.5 tile skipping and 4.2 local attention);
+// the mask is applied only on tiles that straddle the visible band.
 #include <algorithm>
 
 #include "common.cuh"
@@ -67,6 +70,7 @@ struct FwdParams {
   long long o_bstride, lse_bstride, lse_hstride;
   float scale_log2;
   int causal;
+  int win_l, win_r;  // key j visible from row i iff i + diag - win_l <= j <= i + diag + win_r
   int* status;
   long long wait_limit;
 };
@@ -103,10 +107,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int m0 = m_tile * BM;
   if (m0 >= len_q) return;  // uniform: before any barrier or TMEM use
   const int hk = h / (p.Hq / p.Hkv);
-  const int diag = len_k - len_q;  // key j visible from row i iff j <= i + diag
-  int kv_end = len_k;
-  if (p.causal) kv_end = min(len_k, m0 + BM + diag);
-  const int n_kv = kv_end > 0 ? (kv_end + BN - 1) / BN : 0;
+  const int diag = len_k - len_q;  // row i is aligned with key i + diag
+  // keys [kv_begin, kv_end) hold every key visible from rows m0 .. m0 + BM - 1
+  const int kv_end = min(len_k, m0 + BM + diag + p.win_r);
+  const int kv_begin = max(0, m0 + diag - p.win_l);
+  const int j_first = kv_begin / BN;
+  const int n_kv = kv_end > kv_begin ? (kv_end + BN - 1) / BN - j_first : 0;
 
   // ---- setup
   if (threadIdx.x == 0) {
@@ -135,7 +141,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ===================================================== TMA producer
-    if (lane == 0) {
+    // no visible tile: load nothing (no copy may be left in flight at exit)
+    if (lane == 0 && n_kv > 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
@@ -151,13 +158,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_expect_tx(&s.k_full[st], Smem::kTileBytes);
 #pragma unroll
         for (int kb = 0; kb < KB; ++kb)
-          tma_load_4d(s.k[st] + kb * BN * 128, &tm_k, &s.k_full[st], kb * 64, hk, k_off + j * BN, bidx);
+          tma_load_4d(s.k[st] + kb * BN * 128, &tm_k, &s.k_full[st], kb * 64, hk, k_off + (j_first + j) * BN, bidx);
         ++issued_k;
         if (!mbar_wait(&s.v_empty[st], ph ^ 1, ab)) break;
         mbar_expect_tx(&s.v_full[st], Smem::kTileBytes);
 #pragma unroll
         for (int kb = 0; kb < KB; ++kb)
-          tma_load_4d(s.v[st] + kb * BN * 128, &tm_v, &s.v_full[st], kb * 64, hk, k_off + j * BN, bidx);
+          tma_load_4d(s.v[st] + kb * BN * 128, &tm_v, &s.v_full[st], kb * 64, hk, k_off + (j_first + j) * BN, bidx);
         ++issued_v;
       }
       if (s.abort_flag) {
@@ -255,7 +262,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int c = 0; c < 4; ++c) tmem_ld32(tmem + lane_off + kColS + buf * BN + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
       tmem_wait_ld();
       reg_fence(sr);
-      const int kbase = j * BN;
+      const int kbase = (j_first + j) * BN;
       if constexpr (!FAST) {
         // general scores: t = s * scale * log2(e) (+ bias * log2(e))
 #pragma unroll
@@ -266,12 +273,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           sr[c] = __float_as_uint(x);
         }
       }
-      if ((kbase + BN > len_k) || (p.causal && kbase + BN - 1 > m0 + diag)) {
-        // diagonal or ragged tile: hide invisible keys
-        const int lim = min(len_k, p.causal ? i + diag + 1 : len_k) - kbase;
+      if ((kbase + BN > len_k) || (kbase + BN - 1 > m0 + diag + p.win_r) ||
+          (kbase < m0 + BM - 1 + diag - p.win_l)) {
+        // tile on an edge of the visible band, or ragged: hide invisible keys
+        const int hi = min(len_k, i + diag + p.win_r + 1) - kbase;
+        const int lo = i + diag - p.win_l - kbase;
 #pragma unroll
         for (int c = 0; c < BN; ++c)
-          if (c >= lim) sr[c] = 0xff800000u;  // -inf
+          if (c >= hi || c < lo) sr[c] = 0xff800000u;  // -inf
       }
       float mx0 = -INFINITY, mx1 = -INFINITY;
 #pragma unroll
@@ -426,6 +435,8 @@ int launch_fwd_sm100(const TcGeom& g, __nv_bfloat16* o, float* lse, cudaStream_t
   p.lse_hstride = g.Nq;  // packed: Nq is the total row count
   p.scale_log2 = g.scale * kLog2e;
   p.causal = g.causal;
+  p.win_l = win_left(g.window_left);
+  p.win_r = win_right(g.causal, g.window_right);
   p.status = device_status_ptr();
   p.wait_limit = kWaitLimitCycles;
   if (!p.status) return ATTN_ERR_CUDA;

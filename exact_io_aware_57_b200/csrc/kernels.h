@@ -23,12 +23,28 @@ constexpr long long kWaitLimitCycles = 2000000000LL;
 int* device_status_ptr();
 
 // ----------------------------------------------------------------- fp32 path
+// Key visibility.  With a = i + Nk - Nq the key aligned with query row i, key j
+// is visible iff a - win_l <= j <= a + win_r.  kWinNone marks an unbounded side;
+// causal is the right side capped at 0.  Sequence lengths are limited to
+// kMaxSeqLen so that a + kWinNone + 1 and a - kWinNone stay inside int.
+constexpr int kWinNone = 1 << 30;
+constexpr int kMaxSeqLen = 1 << 28;
+inline int win_left(int window_left) {
+  return (window_left < 0 || window_left >= kWinNone) ? kWinNone : window_left;
+}
+inline int win_right(int causal, int window_right) {
+  if (causal) return 0;
+  return (window_right < 0 || window_right >= kWinNone) ? kWinNone : window_right;
+}
+
 struct F32Params {
   const float *q, *k, *v, *bias, *alibi;
   float *o, *lse;
   const int *cu_q, *cu_k;   // packed sequences (device) or null
   long long q_bstride, k_bstride, bias_bstride, lse_bstride, lse_hstride;
   int Hq, Hkv, Nq, Nk, D, causal;
+  int window_left = -1, window_right = -1;  // local attention sizes; negative: unbounded
+  int win_l = kWinNone, win_r = kWinNone;  // folded from causal and the sizes by the launchers
   float scale;
 };
 
@@ -52,6 +68,7 @@ struct TcGeom {
   const float* bias;
   long long bias_bstride;
   const float* alibi;          // per-query-head ALiBi slopes (device) or null
+  int window_left = -1, window_right = -1;  // local attention sizes; negative: unbounded
 };
 
 int launch_fwd_sm100(const TcGeom& g, __nv_bfloat16* o, float* lse, cudaStream_t st);

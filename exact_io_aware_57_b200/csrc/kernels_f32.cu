@@ -40,11 +40,18 @@ ATTN_DEVINL Seq seq_of(const F32Params& p, int z) {
   return s;
 }
 
-// Keys 0 .. n-1 are visible from row i (bottom-right aligned causal mask).
-ATTN_DEVINL int visible(const F32Params& p, const Seq& s, int i) {
-  if (!p.causal) return s.nk;
-  const int last = i + (s.nk - s.nq);
-  return last < 0 ? 0 : min(s.nk, last + 1);
+// Keys lo .. end-1 are visible from row i: with a = i + nk - nq (bottom-right
+// alignment), a - win_l <= j <= a + win_r (causal: win_r = 0).
+struct KeyRange {
+  int lo, end;
+};
+ATTN_DEVINL KeyRange visible(const F32Params& p, const Seq& s, int i) {
+  const int a = i + (s.nk - s.nq);
+  KeyRange r;
+  r.lo = max(0, a - p.win_l);
+  r.end = min(s.nk, a + p.win_r + 1);
+  if (r.end < r.lo) r.end = r.lo;
+  return r;
 }
 
 template <int D>
@@ -65,9 +72,9 @@ __global__ void __launch_bounds__(128) fwd_f32_kernel(F32Params p) {
   }
   const float* brow = p.bias ? p.bias + s.b * p.bias_bstride + ((long long)h * s.nq + i) * s.nk : nullptr;
   const float slope = p.alibi ? p.alibi[h] : 0.f;
-  const int nvis = visible(p, s, i);
+  const KeyRange kr = visible(p, s, i);
   float m = -INFINITY, l = 0.f;
-  for (int j = 0; j < nvis; ++j) {
+  for (int j = kr.lo; j < kr.end; ++j) {
     const long long kv = s.b * p.k_bstride + ((long long)(s.k0 + j) * p.Hkv + hk) * D;
     float dot = 0.f;
 #pragma unroll
@@ -136,8 +143,9 @@ __global__ void __launch_bounds__(128) bwd_dq_f32_kernel(F32Params p, const floa
   }
   const float* brow = p.bias ? p.bias + s.b * p.bias_bstride + ((long long)h * s.nq + i) * s.nk : nullptr;
   const float slope = p.alibi ? p.alibi[h] : 0.f;
-  const int nvis = lse == -INFINITY ? 0 : visible(p, s, i);
-  for (int j = 0; j < nvis; ++j) {
+  KeyRange kr = visible(p, s, i);
+  if (lse == -INFINITY) kr.end = kr.lo;
+  for (int j = kr.lo; j < kr.end; ++j) {
     const long long kv = s.b * p.k_bstride + ((long long)(s.k0 + j) * p.Hkv + hk) * D;
     float dot = 0.f, dpv = 0.f;
 #pragma unroll
@@ -177,13 +185,15 @@ __global__ void __launch_bounds__(128) bwd_dkdv_f32_kernel(F32Params p, const fl
     dka[e] = 0.f;
     dva[e] = 0.f;
   }
-  // row i sees key j iff j <= i + (nk - nq)
-  const int i0 = p.causal ? max(0, j - (s.nk - s.nq)) : 0;
+  // row i sees key j iff j - diag - win_r <= i <= j - diag + win_l
+  const int diag = s.nk - s.nq;
+  const int i0 = max(0, j - diag - p.win_r);
+  const int i_end = min(s.nq, j - diag + p.win_l + 1);
   for (int g = 0; g < G; ++g) {
     const int h = hk * G + g;
     const float* bcol = p.bias ? p.bias + s.b * p.bias_bstride + (long long)h * s.nq * s.nk + j : nullptr;
     const float slope = p.alibi ? p.alibi[h] : 0.f;
-    for (int i = i0; i < s.nq; ++i) {
+    for (int i = i0; i < i_end; ++i) {
       const long long li = s.b * p.lse_bstride + (long long)h * p.lse_hstride + s.q0 + i;
       const float lse = p.lse[li];
       if (lse == -INFINITY) continue;
@@ -215,7 +225,17 @@ __global__ void __launch_bounds__(128) bwd_dkdv_f32_kernel(F32Params p, const fl
 
 }  // namespace
 
-int launch_fwd_f32(const F32Params& p, int num_z, int max_nq, cudaStream_t st) {
+namespace {
+F32Params folded(const F32Params& in) {
+  F32Params p = in;
+  p.win_l = win_left(in.window_left);
+  p.win_r = win_right(in.causal, in.window_right);
+  return p;
+}
+}  // namespace
+
+int launch_fwd_f32(const F32Params& in, int num_z, int max_nq, cudaStream_t st) {
+  const F32Params p = folded(in);
   dim3 grid((max_nq + 3) / 4, p.Hq, num_z);
   if (p.D == 64)
     fwd_f32_kernel<64><<<grid, 128, 0, st>>>(p);
@@ -240,8 +260,9 @@ template int launch_rowdot<float>(const float*, const float*, float*, int, int, 
 template int launch_rowdot<__nv_bfloat16>(const __nv_bfloat16*, const __nv_bfloat16*, float*, int, int, int,
                                           int, cudaStream_t);
 
-int launch_bwd_f32(const F32Params& p, const float* dout, const float* Drow, float* dq, float* dk, float* dv,
+int launch_bwd_f32(const F32Params& in, const float* dout, const float* Drow, float* dq, float* dk, float* dv,
                    int num_z, int max_nq, int max_nk, cudaStream_t st) {
+  const F32Params p = folded(in);
   dim3 gq((max_nq + 3) / 4, p.Hq, num_z), gk((max_nk + 3) / 4, p.Hkv, num_z);
   if (p.D == 64) {
     bwd_dq_f32_kernel<64><<<gq, 128, 0, st>>>(p, dout, Drow, dq);

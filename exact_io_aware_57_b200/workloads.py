@@ -58,9 +58,23 @@ def fwd_flops_pair(nq: int, nk: int, d: int, causal: bool) -> float:
     return 4.0 * nq * nk * d * (0.5 if causal else 1.0)
 
 
-def flops(w: Workload, backward: bool | None = None, lengths=None) -> float:
-    """Forward (+ backward when ``backward``) FLOPs of a whole workload."""
+def window_pairs(n: int, left: int) -> int:
+    """Visible (query, key) pairs of causal self-attention over n tokens when
+    each row also sees at most ``left`` earlier keys."""
+    w = min(int(left), n - 1)
+    # rows 0 .. w-1 see i + 1 keys, the other n - w rows see w + 1
+    return w * (w + 1) // 2 + (n - w) * (w + 1) if n > 0 else 0
+
+
+def flops(w: Workload, backward: bool | None = None, lengths=None, window: int | None = None) -> float:
+    """Forward (+ backward when ``backward``) FLOPs of a whole workload.  With a
+    causal sliding ``window`` (keys i - window .. i) the count is 4*d per
+    visible pair, pairs counted exactly."""
     bwd = w.backward if backward is None else backward
+    if window is not None:
+        assert not w.varlen and w.causal
+        f = 4.0 * w.d * window_pairs(w.n, window) * w.batch * w.h_q
+        return f * (3.5 if bwd else 1.0)
     if w.varlen:
         if lengths is None:
             lengths = synth.varlen_lengths(w.num_seqs, w.len_lo, w.len_hi)

@@ -104,6 +104,29 @@ int attn_bwd_alibi(const void* q, const void* k, const void* v, const float* ali
                    int n_k, int d, float scale, int causal, int dtype, void* stream);
 
 /*
+ * Local (sliding-window) attention, optionally with ALiBi slopes.  With
+ * a = i + n_k - n_q the key aligned with query row i, key j is visible iff
+ *   a - window_left <= j <= a + window_right;
+ * a negative size leaves that side unbounded, and causal != 0 caps the right
+ * side at a (window_right is then ignored).  The kernels load only the key
+ * tiles that meet this band and mask only the tiles on its edges
+ * ("Understanding FlashAttention Pt 1", contents 3.5 and 4.2: tile skipping,
+ * local attention).  Rows with no visible key get O = 0, LSE = -inf.
+ * alibi_slopes: DEVICE fp32 [h_q] or NULL (as attn_fwd_alibi).
+ * Sizes must be at most 2^28 rows per sequence.  Otherwise as attn_fwd.
+ */
+int attn_fwd_local(const void* q, const void* k, const void* v, const float* alibi_slopes, void* o,
+                   float* lse, int batch, int h_q, int h_kv, int n_q, int n_k, int d, float scale,
+                   int causal, int window_left, int window_right, int dtype, void* stream);
+
+/* Backward of attn_fwd_local (same slopes and window); otherwise as attn_bwd. */
+int attn_bwd_local(const void* q, const void* k, const void* v, const float* alibi_slopes,
+                   const void* o, const float* lse, const void* dout, void* dq, void* dk, void* dv,
+                   void* workspace, size_t workspace_bytes, int batch, int h_q, int h_kv, int n_q,
+                   int n_k, int d, float scale, int causal, int window_left, int window_right,
+                   int dtype, void* stream);
+
+/*
  * attn_bwd without a workspace argument, for callers that cannot allocate
  * device memory when they run the backward (code inside a framework that owns
  * all device memory, or latency-critical loops that cannot afford cudaMalloc's

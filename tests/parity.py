@@ -91,7 +91,7 @@ def sample_rows(n: int, tile: int = 128, extra: int = 6, seed: int = 0):
     return sorted(r for r in rows if 0 <= r < n)
 
 
-def check_fwd_sampled(orc, q, k, v, o, lse, causal, heads, rows, bias_fn=None, scale=None):
+def check_fwd_sampled(orc, q, k, v, o, lse, causal, heads, rows, bias_fn=None, scale=None, window=None):
     """Compare sampled outputs of a full-size launch (CPU copies) with the oracle,
     one (batch, head) at a time.  bias_fn(h, rows) -> [R, Nk] fp32 or None."""
     B, Nq, Hq, d = q.shape
@@ -101,7 +101,7 @@ def check_fwd_sampled(orc, q, k, v, o, lse, causal, heads, rows, bias_fn=None, s
     for (b, h) in heads:
         br = bias_fn(h, rows) if bias_fn else None
         o_ref, l_ref = orc.fwd_rows(q[b, rows, h], k[b, :, h // G], v[b, :, h // G], rows, Nq, bias_rows=br,
-                                    causal=causal, scale=scale)
+                                    causal=causal, scale=scale, window=window)
         worst_o = max(worst_o, max_abs(o[b, rows, h].double().numpy(), o_ref))
         worst_l = max(worst_l, max_abs(lse[b, h, rows].double().numpy(), l_ref))
     return worst_o, worst_l
