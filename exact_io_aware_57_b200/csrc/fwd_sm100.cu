@@ -38,7 +38,9 @@ namespace {
 
 constexpr int BM = 128;          // query rows per CTA
 constexpr int BN = 128;          // keys per KV tile
-constexpr int NST = 2;           // K/V smem stages
+// K/V shared-memory stages: as many as fit beside the Q tile in 227 KB
+template <int D>
+constexpr int kStages = D == 64 ? 4 : 3;
 constexpr int kThreads = 192;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColO = 256, kColP = 384;
@@ -46,6 +48,7 @@ constexpr float kRescaleThreshold = 8.f;  // log2 units: P stays <= 256
 
 template <int D>
 struct FwdSmem {
+  static constexpr int NST = kStages<D>;
   static constexpr int kTileBytes = BM * D * 2;  // 128 rows x D bf16
   alignas(1024) uint8_t q[kTileBytes];
   alignas(1024) uint8_t k[NST][kTileBytes];
@@ -87,6 +90,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
   using Smem = FwdSmem<D>;
+  constexpr int NST = Smem::NST;
   constexpr int KB = D / 64;  // 64-column (128-byte) blocks per row
   extern __shared__ uint8_t smem_raw[];
   Smem& s = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
