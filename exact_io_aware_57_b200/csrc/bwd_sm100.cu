@@ -21,11 +21,18 @@
 // TMEM columns: [0,128) S^T (then P^T as bf16 pairs in [0,64)),
 //   [128,256) dP^T (then the dQ tile), [256,256+D) dV, [256+D,256+2D) dK.
 // Per step (query head h, query tile i):
-//   MMA   S^T = K_j Q_i^T;  dP^T = V_j dO_i^T (once the previous dQ left TMEM)
+//   MMA   S^T = K_j Q_i^T and dP^T = V_j dO_i^T, interleaved (once the previous
+//         dQ has left TMEM)
 //   WG0   P^T = 2^(scale log2e S^T + log2e B^T - log2e LSE) -> TMEM (bf16);
 //         dS^T = P^T o (dP^T - D) -> shared memory (bf16, 128B-swizzled)
-//   MMA   dK += dS^T Q_i and dQ_i = dS K_j, then dV += P^T dO_i (P^T from TMEM)
-//   WG1   dQ_i -> shared memory -> TMA bulk reduce-add into the fp32 accumulator
+//   MMA   dV += P^T dO_i (P^T from TMEM), dK += dS^T Q_i and dQ_i = dS K_j,
+//         interleaved
+//   WG1   dQ_i -> the step's own Q_i/dO_i buffers (free once its MMAs are done)
+//         -> TMA bulk reduce-add into the fp32 accumulator; the producer
+//         refills those buffers only after the reduction has read them, so the
+//         reduction overlaps the next step instead of holding up its dS^T.
+// A chain of MMAs into one TMEM accumulator waits on each previous result;
+// every group above interleaves two or three accumulators instead.
 #include <algorithm>
 
 #include "common.cuh"
@@ -52,8 +59,8 @@ struct BwdSmem {
   alignas(1024) uint8_t ds[128 * 128 * 2];  // dS^T, [key][query] in two 64-column blocks
   alignas(16) float nlse2[NSTQ][BM];        // -log2(e) * LSE of the step's query rows (-inf: no key)
   alignas(16) float drow[NSTQ][BM];         // D_i of the step's query rows
-  uint64_t kv_full, q_full[NSTQ], q_empty[NSTQ];
-  uint64_t st_full, dpt_full, ds_ready, dkq_done, tmem_free, staging_free, drain;
+  uint64_t kv_full, q_full[NSTQ], q_free[NSTQ];
+  uint64_t st_full, ds_ready, dkq_done, tmem_free, drain;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -105,85 +112,114 @@ ATTN_DEVINL void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
 // bf16 pairs over the S^T columns already read (A operand of dV += P^T dO).
 // MASK zeroes queries this key is hidden from (query i sees key kj iff
 // kj - lo_off <= i <= kj + hi_off, i.e. i + diag - win_l <= kj <= i + diag + win_r;
-// padding rows and keys).  Rolled over chunks so the code stays small enough
-// for the instruction cache.
+// padding rows and keys).
+template <bool MASK, int BIAS>
+ATTN_DEVINL void p_chunk(int c, const uint32_t (&sr)[32], uint32_t st_col, const float* nlse2, float scale_log2,
+                         const float* bcol, float neg_slope2, int nk, int i0, int len_q, int kj, int len_k,
+                         int lo_off, int hi_off, int bias_diag) {
+  const float4* nl4 = reinterpret_cast<const float4*>(nlse2 + c * 32);
+  const int q0 = i0 + c * 32;
+  int vis_lo = 0, vis_hi = 32;  // queries q0 + e, vis_lo <= e < vis_hi, see this key
+  if constexpr (MASK) {
+    vis_lo = kj - lo_off - q0;
+    vis_hi = min(min(32, len_q - q0), kj + hi_off - q0 + 1);
+    if (kj >= len_k) vis_hi = 0;
+  }
+  uint32_t pk[16];
+#pragma unroll
+  for (int e4 = 0; e4 < 8; ++e4) {
+    const float4 nl = nl4[e4];
+    const float nlv[4] = {nl.x, nl.y, nl.z, nl.w};
+    float pv[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int e = e4 * 4 + u;
+      float t = fmaf(__uint_as_float(sr[e]), scale_log2, nlv[u]);
+      if constexpr (BIAS == kBiasDense) t = fmaf(__ldg(bcol + (long long)min(q0 + e, len_q - 1) * nk), kLog2e, t);
+      if constexpr (BIAS == kBiasAlibi) t = fmaf(neg_slope2, fabsf(static_cast<float>(kj - q0 - e - bias_diag)), t);
+      float pe = ex2(t);
+      if constexpr (MASK) pe = (e >= vis_lo && e < vis_hi) ? pe : 0.f;
+      pv[u] = pe;
+    }
+    pk[2 * e4] = pack_bf16(pv[0], pv[1]);
+    pk[2 * e4 + 1] = pack_bf16(pv[2], pv[3]);
+  }
+  tmem_st16(st_col + c * 16, pk);  // columns [16c, 16c+16): S^T there is already read
+}
+
+// The four chunks with the TMEM load of the next chunk in flight while one is
+// computed (the P^T store of chunk c lands on columns of chunks <= c, all read).
 template <bool MASK, int BIAS>
 ATTN_DEVINL void bwd_p_chunks(uint32_t st_col, const float* nlse2, float scale_log2, const float* bcol,
                               float neg_slope2, int nk, int i0, int len_q, int kj, int len_k, int lo_off,
                               int hi_off, int bias_diag) {
+  uint32_t ra[32], rb[32];
+  tmem_ld32(st_col, ra);
 #pragma unroll 1
-  for (int c = 0; c < BM / 32; ++c) {
-    uint32_t sr[32];
-    tmem_ld32(st_col + c * 32, sr);
+  for (int c = 0; c < BM / 32; c += 2) {
     tmem_wait_ld();
-    reg_fence(sr);
-    const float4* nl4 = reinterpret_cast<const float4*>(nlse2 + c * 32);
-    const int q0 = i0 + c * 32;
-    int vis_lo = 0, vis_hi = 32;  // queries q0 + e, vis_lo <= e < vis_hi, see this key
-    if constexpr (MASK) {
-      vis_lo = kj - lo_off - q0;
-      vis_hi = min(min(32, len_q - q0), kj + hi_off - q0 + 1);
-      if (kj >= len_k) vis_hi = 0;
-    }
-    uint32_t pk[16];
-#pragma unroll
-    for (int e4 = 0; e4 < 8; ++e4) {
-      const float4 nl = nl4[e4];
-      const float nlv[4] = {nl.x, nl.y, nl.z, nl.w};
-      float pv[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int e = e4 * 4 + u;
-        float t = fmaf(__uint_as_float(sr[e]), scale_log2, nlv[u]);
-        if constexpr (BIAS == kBiasDense) t = fmaf(__ldg(bcol + (long long)min(q0 + e, len_q - 1) * nk), kLog2e, t);
-        if constexpr (BIAS == kBiasAlibi)
-          t = fmaf(neg_slope2, fabsf(static_cast<float>(kj - q0 - e - bias_diag)), t);
-        float pe = ex2(t);
-        if constexpr (MASK) pe = (e >= vis_lo && e < vis_hi) ? pe : 0.f;
-        pv[u] = pe;
-      }
-      pk[2 * e4] = pack_bf16(pv[0], pv[1]);
-      pk[2 * e4 + 1] = pack_bf16(pv[2], pv[3]);
-    }
-    tmem_st16(st_col + c * 16, pk);  // columns [16c, 16c+16): S^T there is already read
+    reg_fence(ra);
+    tmem_ld32(st_col + (c + 1) * 32, rb);
+    p_chunk<MASK, BIAS>(c, ra, st_col, nlse2, scale_log2, bcol, neg_slope2, nk, i0, len_q, kj, len_k, lo_off,
+                        hi_off, bias_diag);
+    tmem_wait_ld();
+    reg_fence(rb);
+    if (c + 2 < BM / 32) tmem_ld32(st_col + (c + 2) * 32, ra);
+    p_chunk<MASK, BIAS>(c + 1, rb, st_col, nlse2, scale_log2, bcol, neg_slope2, nk, i0, len_q, kj, len_k, lo_off,
+                        hi_off, bias_diag);
   }
 }
 
 // Phase B -- dS^T = P^T (dP^T - D) from the bf16 P^T in TMEM and dP^T, into the
 // 128B-swizzled shared tile (K-major for dK += dS^T Q, MN-major for dQ = dS K).
-ATTN_DEVINL void bwd_ds_chunks(uint32_t st_col, uint32_t dp_col, const float* drow, uint32_t ds_row, int r) {
-#pragma unroll 1
-  for (int c = 0; c < BM / 32; ++c) {
-    uint32_t pr[16], dpr[32];
-    tmem_ld16(st_col + c * 16, pr);
-    tmem_ld32(dp_col + c * 32, dpr);
-    tmem_wait_ld();
-    reg_fence(pr);
-    reg_fence(dpr);
-    const float4* dr4 = reinterpret_cast<const float4*>(drow + c * 32);
-    uint32_t dk[16];
+ATTN_DEVINL void ds_chunk(int c, const uint32_t (&pr)[16], const uint32_t (&dpr)[32], const float* drow,
+                          uint32_t ds_row, int r) {
+  const float4* dr4 = reinterpret_cast<const float4*>(drow + c * 32);
+  uint32_t dk[16];
 #pragma unroll
-    for (int e4 = 0; e4 < 8; ++e4) {
-      const float4 dr = dr4[e4];
-      const float drv[4] = {dr.x, dr.y, dr.z, dr.w};
-      float dsv[4];
-#pragma unroll
-      for (int u = 0; u < 4; ++u) {
-        const int e = e4 * 4 + u;
-        const uint32_t pair = pr[e >> 1];
-        const float pe = __uint_as_float((e & 1) ? (pair & 0xffff0000u) : (pair << 16));
-        dsv[u] = pe * (__uint_as_float(dpr[e]) - drv[u]);
-      }
-      dk[2 * e4] = pack_bf16(dsv[0], dsv[1]);
-      dk[2 * e4 + 1] = pack_bf16(dsv[2], dsv[3]);
-    }
-    // 32 queries = 4 chunks of 16 bytes in 64-column block c/2
+  for (int e4 = 0; e4 < 8; ++e4) {
+    const float4 dr = dr4[e4];
+    const float drv[4] = {dr.x, dr.y, dr.z, dr.w};
+    float dsv[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const int chunk = (c & 1) * 4 + u;  // 16-byte chunk within the 128-byte row
-      const uint32_t addr = ds_row + (c >> 1) * (128 * 128) + ((chunk ^ (r & 7)) << 4);
-      st_shared_v4(addr, dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
+      const int e = e4 * 4 + u;
+      const uint32_t pair = pr[e >> 1];
+      const float pe = __uint_as_float((e & 1) ? (pair & 0xffff0000u) : (pair << 16));
+      dsv[u] = pe * (__uint_as_float(dpr[e]) - drv[u]);
     }
+    dk[2 * e4] = pack_bf16(dsv[0], dsv[1]);
+    dk[2 * e4 + 1] = pack_bf16(dsv[2], dsv[3]);
+  }
+  // 32 queries = 4 chunks of 16 bytes in 64-column block c/2
+#pragma unroll
+  for (int u = 0; u < 4; ++u) {
+    const int chunk = (c & 1) * 4 + u;  // 16-byte chunk within the 128-byte row
+    const uint32_t addr = ds_row + (c >> 1) * (128 * 128) + ((chunk ^ (r & 7)) << 4);
+    st_shared_v4(addr, dk[4 * u], dk[4 * u + 1], dk[4 * u + 2], dk[4 * u + 3]);
+  }
+}
+
+ATTN_DEVINL void bwd_ds_chunks(uint32_t st_col, uint32_t dp_col, const float* drow, uint32_t ds_row, int r) {
+  uint32_t pa[16], da[32], pb[16], db[32];
+  tmem_ld16(st_col, pa);
+  tmem_ld32(dp_col, da);
+#pragma unroll 1
+  for (int c = 0; c < BM / 32; c += 2) {
+    tmem_wait_ld();
+    reg_fence(pa);
+    reg_fence(da);
+    tmem_ld16(st_col + (c + 1) * 16, pb);
+    tmem_ld32(dp_col + (c + 1) * 32, db);
+    ds_chunk(c, pa, da, drow, ds_row, r);
+    tmem_wait_ld();
+    reg_fence(pb);
+    reg_fence(db);
+    if (c + 2 < BM / 32) {
+      tmem_ld16(st_col + (c + 2) * 16, pa);
+      tmem_ld32(dp_col + (c + 2) * 32, da);
+    }
+    ds_chunk(c + 1, pb, db, drow, ds_row, r);
   }
 }
 
@@ -220,14 +256,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&s.kv_full, 1);
     for (int i = 0; i < NSTQ; ++i) {
       mbar_init(&s.q_full[i], 1 + 32);  // TMA transaction arrive + 32 producer lanes (LSE/D rows)
-      mbar_init(&s.q_empty[i], 1);
+      mbar_init(&s.q_free[i], 1);
     }
     mbar_init(&s.st_full, 1);
-    mbar_init(&s.dpt_full, 1);
     mbar_init(&s.ds_ready, 4);
     mbar_init(&s.dkq_done, 1);
     mbar_init(&s.tmem_free, 4);
-    mbar_init(&s.staging_free, 1);
     mbar_init(&s.drain, 1);
     fence_mbar_init();
   }
@@ -260,7 +294,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t ph = (step / NSTQ) & 1;
       const int h = hk * G + step / per_head;
       const int i0 = (i_first + step % per_head) * BM;
-      const bool ok = __all_sync(0xffffffffu, mbar_wait(&s.q_empty[st], ph ^ 1, ab));
+      // the stage's buffers last held the dQ tile of step - NSTQ: wait until its
+      // reduction has read them
+      const bool ok = __all_sync(0xffffffffu, mbar_wait(&s.q_free[st], ph ^ 1, ab));
       if (!ok) break;
       if (lane == 0) {
         mbar_expect_tx(&s.q_full[st], 2 * Smem::kTileBytes);
@@ -303,46 +339,40 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int step = 0; ok && step < n_steps; ++step) {
         const int st = step % NSTQ;
         if (!mbar_wait(&s.q_full[st], (step / NSTQ) & 1, ab)) break;
+        // dP^T goes where dQ of the previous step was
+        if (step > 0 && !mbar_wait(&s.tmem_free, (step - 1) & 1, ab)) break;
         tc_fence_after();
         const uint32_t q_addr = smem_u32(s.q[st]), do_addr = smem_u32(s.dout[st]);
-        // S^T = K_j Q_i^T.  It overwrites P^T of the previous step, whose dV MMA
-        // was issued earlier by this thread (tcgen05.mma executes in issue order).
+        // S^T = K_j Q_i^T (over P^T of the previous step, whose dV MMA was issued
+        // earlier by this thread: tcgen05.mma executes in issue order) and
+        // dP^T = V_j dO_i^T, round-robin
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
           mma_ss(tmem + kColST, sdesc_sw128(k_addr + off, 16, 1024), sdesc_sw128(q_addr + off, 16, 1024), idesc_s,
                  kk > 0);
-        }
-        mma_commit(&s.st_full);
-        // dP^T = V_j dO_i^T goes where dQ of the previous step was
-        if (step > 0 && !mbar_wait(&s.tmem_free, (step - 1) & 1, ab)) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
           mma_ss(tmem + kColDPT, sdesc_sw128(v_addr + off, 16, 1024), sdesc_sw128(do_addr + off, 16, 1024),
                  idesc_s, kk > 0);
         }
-        mma_commit(&s.dpt_full);
+        // its completion also implies that the previous step's MMAs, the last
+        // readers of the dS^T tile, are done
+        mma_commit(&s.st_full);
         if (!mbar_wait(&s.ds_ready, step & 1, ab)) break;
         tc_fence_after();
-        // dK += dS^T Q_i and dQ_i = dS K_j (the dS^T tile read MN-major), issued
-        // round-robin; their commit releases the dS^T tile to the dQ drain
+        // dV += P^T dO_i (P^T from TMEM), dK += dS^T Q_i and dQ_i = dS K_j (the
+        // dS^T tile read MN-major), round-robin
 #pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk) {
           const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+          mma_ts(tmem + kColDV, tmem + kColST + kk * 8, sdesc_sw128(do_addr + kk * 2048, BM * 128, 1024), idesc_kv,
+                 (step > 0 || kk > 0));
           mma_ss(tmem + kColDK, sdesc_sw128(ds_addr + off, 16, 1024), sdesc_sw128(q_addr + kk * 2048, BM * 128, 1024),
                  idesc_kv, (step > 0 || kk > 0));
           mma_ss(tmem + kColDPT, sdesc_sw128(ds_addr + kk * 2048, 128 * 128, 1024),
                  sdesc_sw128(k_addr + kk * 2048, BN * 128, 1024), idesc_dq, kk > 0);
         }
+        // every MMA of the step is done: dQ_i may leave TMEM and Q_i/dO_i are free
         mma_commit(&s.dkq_done);
-        // dV += P^T dO_i (P^T from TMEM)
-#pragma unroll
-        for (int kk = 0; kk < BM / 16; ++kk)
-          mma_ts(tmem + kColDV, tmem + kColST + kk * 8, sdesc_sw128(do_addr + kk * 2048, BM * 128, 1024), idesc_kv,
-                 (step > 0 || kk > 0));
-        mma_commit(&s.q_empty[st]);
       }
       mma_commit(&s.drain);
       mbar_wait_drain(&s.drain, 0, p.wait_limit);
@@ -359,9 +389,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int st = step % NSTQ;
       const int h = hk * G + step / per_head;
       const int i0 = (i_first + step % per_head) * BM;
+      // S^T and dP^T are in TMEM, and the previous step's MMAs have released the
+      // dS^T tile; q_full of this stage (LSE/D rows) completed before
       ok = __all_sync(0xffffffffu, mbar_wait(&s.st_full, step & 1, ab));
       if (!ok) break;
-      // q_full for this stage (LSE/D rows) completed before st_full
       tc_fence_after();
       // tile-level (warp-uniform) condition: the chunk routines hold
       // warp-collective tcgen05 instructions, so every lane must take the same one
@@ -379,11 +410,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         bwd_p_chunks<false, BIAS>(st_col, s.nlse2[st], p.scale_log2, bcol, neg_slope2, p.Nk, i0, len_q, kj, len_k,
                                   0, 0, diag);
       tmem_wait_st();
-      // dS^T needs dP^T, and the shared tile back from the previous dQ drain
-      ok = __all_sync(0xffffffffu, mbar_wait(&s.dpt_full, step & 1, ab) &&
-                                       (step == 0 || mbar_wait(&s.staging_free, (step - 1) & 1, ab)));
-      if (!ok) break;
-      tc_fence_after();
       bwd_ds_chunks(st_col, dp_col, s.drow[st], ds_row, r);
       fence_proxy_async_smem();
       tc_fence_before();
@@ -427,16 +453,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // ===================================================== dQ drain (thread = query row)
     // dQ_i is read out of TMEM at once (freeing its columns for the next dP^T),
-    // staged through the dS^T shared tile, 64 columns per pass, and added to the
-    // fp32 accumulator by TMA bulk reductions that overlap the next step.
+    // staged through the step's own Q_i / dO_i buffers -- four 128-row x 32-column
+    // fp32 boxes, 128B-swizzled like the TMA map -- and added to the fp32
+    // accumulator by TMA bulk reductions; the producer refills the buffers once
+    // the reductions have read them.
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const bool leader = warp == 6 && lane == 0;
-    const uint32_t stage_row = smem_u32(s.ds) + r * 128;
     for (int step = 0; step < n_steps; ++step) {
+      const int st = step % NSTQ;
       const int h = hk * G + step / per_head;
       const int i0 = (i_first + step % per_head) * BM;
+      // every MMA of the step is done: dQ_i is final and Q_i / dO_i are unused
       if (!__all_sync(0xffffffffu, mbar_wait(&s.dkq_done, step & 1, ab))) break;
       tc_fence_after();
       uint32_t a[D];
@@ -447,35 +476,28 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s.tmem_free);
+      // box c (columns 32c .. 32c+31, 16 KB): each buffer holds D / 64 boxes,
+      // Q_i's first, then dO_i's
+      constexpr int kBoxes = D / 64;
+      const uint32_t q_row = smem_u32(s.q[st]) + r * 128, do_row = smem_u32(s.dout[st]) + r * 128;
 #pragma unroll
-      for (int pass = 0; pass < D / 64; ++pass) {
-        if (pass > 0) {
-          if (leader) bulk_wait_read0();  // the previous pass's reductions have read the tile
-          __syncwarp();
-          named_bar_sync(1, 128);
+      for (int c = 0; c < D / 32; ++c) {
+        const uint32_t row = (c < kBoxes ? q_row : do_row) + (c % kBoxes) * (128 * 128);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int e = c * 32 + 4 * u;
+          st_shared_v4(row + ((u ^ (r & 7)) << 4), a[e], a[e + 1], a[e + 2], a[e + 3]);
         }
-        // 2 x 32 fp32 = 2 x 8 chunks of 16 bytes, 128B-swizzled like the TMA box
-#pragma unroll
-        for (int cc = 0; cc < 2; ++cc)
-#pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            const int e = (pass * 2 + cc) * 32 + 4 * u;
-            st_shared_v4(stage_row + cc * (128 * 128) + ((u ^ (r & 7)) << 4), a[e], a[e + 1], a[e + 2], a[e + 3]);
-          }
-        fence_proxy_async_smem();
-        named_bar_sync(1, 128);
-        if (leader) {
-#pragma unroll
-          for (int cc = 0; cc < 2; ++cc)
-            tma_reduce_add_4d(&tm_dq, s.ds + cc * (128 * 128), (pass * 2 + cc) * 32, h, i0, b);
-          bulk_commit();
-        }
-        __syncwarp();
       }
-      // the next step's dS^T overwrites the staging tile: hand it back once read
+      fence_proxy_async_smem();
+      named_bar_sync(1, 128);
       if (leader) {
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c)
+          tma_reduce_add_4d(&tm_dq, (c < kBoxes ? s.q[st] : s.dout[st]) + (c % kBoxes) * (128 * 128), c * 32, h, i0, b);
+        bulk_commit();
         bulk_wait_read0();
-        mbar_arrive(&s.staging_free);
+        mbar_arrive(&s.q_free[st]);
       }
       __syncwarp();
     }
