@@ -14,23 +14,27 @@
 //   bwd_dq     dQ = scale * accumulator -> bf16
 //
 // bwd_main roles (10 warps):
-//   warp 0      TMA producer (K_j, V_j once; Q_i, dO_i per step) + LSE/D rows
+//   warp 0      TMA producer (K_j, V_j once; Q_i, dO_i per step) + LSE/D rows,
+//               and the TMA reduce-add of each staged dQ tile
 //   warp 1      TMEM owner + single-thread tcgen05.mma issuer
-//   warps 2..5  thread t owns key row t: P^T, dS^T, and the dK/dV epilogue
-//   warps 6..9  thread t owns query row t of the dQ tile: TMEM -> smem -> TMA reduce-add
+//   warps 2..9  two groups of four; TMEM lane t is key row t for P^T / dS^T and
+//               the dK/dV epilogue, and query row t for the dQ tile.  Group g
+//               takes queries [64g, 64g+64) of P^T / dS^T and columns
+//               [gD/2, (g+1)D/2) of dQ, dK and dV, so every SM sub-partition
+//               runs two warps of each elementwise phase.
 // TMEM columns: [0,128) S^T (then P^T as bf16 pairs in [0,64)),
 //   [128,256) dP^T (then the dQ tile), [256,256+D) dV, [256+D,256+2D) dK.
 // Per step (query head h, query tile i):
 //   MMA   S^T = K_j Q_i^T and dP^T = V_j dO_i^T, interleaved (once the previous
 //         dQ has left TMEM)
-//   WG0   P^T = 2^(scale log2e S^T + log2e B^T - log2e LSE) -> TMEM (bf16);
+//   WGs   P^T = 2^(scale log2e S^T + log2e B^T - log2e LSE) -> TMEM (bf16);
 //         dS^T = P^T o (dP^T - D) -> shared memory (bf16, 128B-swizzled)
 //   MMA   dV += P^T dO_i (P^T from TMEM), dK += dS^T Q_i and dQ_i = dS K_j,
 //         interleaved
-//   WG1   dQ_i -> the step's own Q_i/dO_i buffers (free once its MMAs are done)
-//         -> TMA bulk reduce-add into the fp32 accumulator; the producer
-//         refills those buffers only after the reduction has read them, so the
-//         reduction overlaps the next step instead of holding up its dS^T.
+//   WGs   dQ_i -> the step's own Q_i/dO_i buffers (free once its MMAs are done);
+//         the producer adds them into the fp32 accumulator with TMA bulk
+//         reductions and refills the buffers only after those have read them,
+//         so the reduction overlaps the next step instead of holding it up.
 // A chain of MMAs into one TMEM accumulator waits on each previous result;
 // every group above interleaves two or three accumulators instead.
 #include <algorithm>
@@ -59,8 +63,8 @@ struct BwdSmem {
   alignas(1024) uint8_t ds[128 * 128 * 2];  // dS^T, [key][query] in two 64-column blocks
   alignas(16) float nlse2[NSTQ][BM];        // -log2(e) * LSE of the step's query rows (-inf: no key)
   alignas(16) float drow[NSTQ][BM];         // D_i of the step's query rows
-  uint64_t kv_full, q_full[NSTQ], q_free[NSTQ];
-  uint64_t st_full, ds_ready, dkq_done, tmem_free, drain;
+  uint64_t kv_full, q_full[NSTQ], staged[NSTQ];
+  uint64_t st_full, s_read, ds_ready, dkq_done, tmem_free, drain;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -100,8 +104,6 @@ ATTN_DEVINL void tma_reduce_add_4d(const CUtensorMap* map, const void* src, int 
 ATTN_DEVINL void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 ATTN_DEVINL void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 ATTN_DEVINL void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-// non-.aligned form: legal even if the calling warp arrives diverged
-ATTN_DEVINL void named_bar_sync(int id, int n) { asm volatile("barrier.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
 
 ATTN_DEVINL void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
   asm volatile("st.shared.v4.b32 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
@@ -147,27 +149,34 @@ ATTN_DEVINL void p_chunk(int c, const uint32_t (&sr)[32], uint32_t st_col, const
   tmem_st16(st_col + c * 16, pk);  // columns [16c, 16c+16): S^T there is already read
 }
 
-// The four chunks with the TMEM load of the next chunk in flight while one is
-// computed (the P^T store of chunk c lands on columns of chunks <= c, all read).
+// Group g's half of phase A: queries [64g, 64g+64), chunks 2g and 2g+1.  The
+// P^T of group 1 lands on S^T columns [32, 64), which group 0 reads: group 0's
+// warps arrive on `s_read` once their loads are complete and group 1 waits for
+// that phase (bounded) before it stores.  Returns false if that wait gave up.
 template <bool MASK, int BIAS>
-ATTN_DEVINL void bwd_p_chunks(uint32_t st_col, const float* nlse2, float scale_log2, const float* bcol,
-                              float neg_slope2, int nk, int i0, int len_q, int kj, int len_k, int lo_off,
-                              int hi_off, int bias_diag) {
+ATTN_DEVINL bool bwd_p_half(int grp, uint64_t* s_read, uint32_t parity, const Abort& ab, uint32_t st_col,
+                            const float* nlse2, float scale_log2, const float* bcol, float neg_slope2, int nk, int i0,
+                            int len_q, int kj, int len_k, int lo_off, int hi_off, int bias_diag) {
+  const int c0 = 2 * grp;
   uint32_t ra[32], rb[32];
-  tmem_ld32(st_col, ra);
-#pragma unroll 1
-  for (int c = 0; c < BM / 32; c += 2) {
-    tmem_wait_ld();
-    reg_fence(ra);
-    tmem_ld32(st_col + (c + 1) * 32, rb);
-    p_chunk<MASK, BIAS>(c, ra, st_col, nlse2, scale_log2, bcol, neg_slope2, nk, i0, len_q, kj, len_k, lo_off,
-                        hi_off, bias_diag);
-    tmem_wait_ld();
-    reg_fence(rb);
-    if (c + 2 < BM / 32) tmem_ld32(st_col + (c + 2) * 32, ra);
-    p_chunk<MASK, BIAS>(c + 1, rb, st_col, nlse2, scale_log2, bcol, neg_slope2, nk, i0, len_q, kj, len_k, lo_off,
-                        hi_off, bias_diag);
+  tmem_ld32(st_col + c0 * 32, ra);
+  tmem_ld32(st_col + (c0 + 1) * 32, rb);
+  tmem_wait_ld();
+  reg_fence(ra);
+  reg_fence(rb);
+  if (grp == 0) {
+    tc_fence_before();
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(s_read);
+  } else {
+    if (!__all_sync(0xffffffffu, mbar_wait(s_read, parity, ab))) return false;
+    tc_fence_after();
   }
+  p_chunk<MASK, BIAS>(c0, ra, st_col, nlse2, scale_log2, bcol, neg_slope2, nk, i0, len_q, kj, len_k, lo_off, hi_off,
+                      bias_diag);
+  p_chunk<MASK, BIAS>(c0 + 1, rb, st_col, nlse2, scale_log2, bcol, neg_slope2, nk, i0, len_q, kj, len_k, lo_off,
+                      hi_off, bias_diag);
+  return true;
 }
 
 // Phase B -- dS^T = P^T (dP^T - D) from the bf16 P^T in TMEM and dP^T, into the
@@ -200,27 +209,21 @@ ATTN_DEVINL void ds_chunk(int c, const uint32_t (&pr)[16], const uint32_t (&dpr)
   }
 }
 
-ATTN_DEVINL void bwd_ds_chunks(uint32_t st_col, uint32_t dp_col, const float* drow, uint32_t ds_row, int r) {
+// Group g's half of phase B (its own P^T columns, chunks 2g and 2g+1).
+ATTN_DEVINL void bwd_ds_half(int grp, uint32_t st_col, uint32_t dp_col, const float* drow, uint32_t ds_row, int r) {
+  const int c0 = 2 * grp;
   uint32_t pa[16], da[32], pb[16], db[32];
-  tmem_ld16(st_col, pa);
-  tmem_ld32(dp_col, da);
-#pragma unroll 1
-  for (int c = 0; c < BM / 32; c += 2) {
-    tmem_wait_ld();
-    reg_fence(pa);
-    reg_fence(da);
-    tmem_ld16(st_col + (c + 1) * 16, pb);
-    tmem_ld32(dp_col + (c + 1) * 32, db);
-    ds_chunk(c, pa, da, drow, ds_row, r);
-    tmem_wait_ld();
-    reg_fence(pb);
-    reg_fence(db);
-    if (c + 2 < BM / 32) {
-      tmem_ld16(st_col + (c + 2) * 16, pa);
-      tmem_ld32(dp_col + (c + 2) * 32, da);
-    }
-    ds_chunk(c + 1, pb, db, drow, ds_row, r);
-  }
+  tmem_ld16(st_col + c0 * 16, pa);
+  tmem_ld32(dp_col + c0 * 32, da);
+  tmem_ld16(st_col + (c0 + 1) * 16, pb);
+  tmem_ld32(dp_col + (c0 + 1) * 32, db);
+  tmem_wait_ld();
+  reg_fence(pa);
+  reg_fence(da);
+  reg_fence(pb);
+  reg_fence(db);
+  ds_chunk(c0, pa, da, drow, ds_row, r);
+  ds_chunk(c0 + 1, pb, db, drow, ds_row, r);
 }
 
 template <int D, int BIAS>
@@ -256,12 +259,13 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&s.kv_full, 1);
     for (int i = 0; i < NSTQ; ++i) {
       mbar_init(&s.q_full[i], 1 + 32);  // TMA transaction arrive + 32 producer lanes (LSE/D rows)
-      mbar_init(&s.q_free[i], 1);
+      mbar_init(&s.staged[i], 8);   // the eight elementwise warps, dQ tile staged
     }
     mbar_init(&s.st_full, 1);
-    mbar_init(&s.ds_ready, 4);
+    mbar_init(&s.s_read, 4);
+    mbar_init(&s.ds_ready, 8);
     mbar_init(&s.dkq_done, 1);
-    mbar_init(&s.tmem_free, 4);
+    mbar_init(&s.tmem_free, 8);
     mbar_init(&s.drain, 1);
     fence_mbar_init();
   }
@@ -272,14 +276,36 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = s.tmem_base;
   const Abort ab{&s.abort_flag, p.status, p.wait_limit};
 
+  constexpr int kBoxes = D / 64;  // 16 KB fp32 dQ boxes (128 rows x 32 columns) per Q or dO buffer
   if (warp == 0) {
     // ===================================================== producer
-    int issued = 0;
+    // Stage st of step s held the dQ tile of step s - NSTQ: before reloading
+    // it, add that tile into the accumulator and wait until the reduction has
+    // read the buffers.
+    int issued = 0, reduced = 0;
+    auto reduce_step = [&](int t) -> bool {
+      const int st = t % NSTQ;
+      if (!__all_sync(0xffffffffu, mbar_wait(&s.staged[st], (t / NSTQ) & 1, ab))) return false;
+      if (lane == 0) {
+        const int h = hk * G + t / per_head;
+        const int i0 = (i_first + t % per_head) * BM;
+#pragma unroll
+        for (int c = 0; c < D / 32; ++c)
+          tma_reduce_add_4d(&tm_dq, (c < kBoxes ? s.q[st] : s.dout[st]) + (c % kBoxes) * (128 * 128), c * 32, h,
+                            i0, b);
+        bulk_commit();
+        bulk_wait_read0();
+      }
+      __syncwarp();
+      ++reduced;
+      return true;
+    };
     if (lane == 0) {
       tma_prefetch_desc(&tm_q);
       tma_prefetch_desc(&tm_k);
       tma_prefetch_desc(&tm_v);
       tma_prefetch_desc(&tm_do);
+      tma_prefetch_desc(&tm_dq);
       if (n_steps > 0) {
         mbar_expect_tx(&s.kv_full, 2 * Smem::kTileBytes);
 #pragma unroll
@@ -289,15 +315,27 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
+    bool ok = true;
     for (int step = 0; step < n_steps; ++step) {
       const int st = step % NSTQ;
-      const uint32_t ph = (step / NSTQ) & 1;
       const int h = hk * G + step / per_head;
       const int i0 = (i_first + step % per_head) * BM;
-      // the stage's buffers last held the dQ tile of step - NSTQ: wait until its
-      // reduction has read them
-      const bool ok = __all_sync(0xffffffffu, mbar_wait(&s.q_free[st], ph ^ 1, ab));
-      if (!ok) break;
+      // LSE / D rows of this step into registers first (their latency overlaps
+      // the wait for the stage)
+      const long long row0 = ((long long)b * p.Hq + h) * p.Nq;
+      float l2v[BM / 32], drv[BM / 32];
+#pragma unroll
+      for (int e = 0; e < BM / 32; ++e) {
+        const int qi = i0 + lane + 32 * e;
+        l2v[e] = -INFINITY;
+        drv[e] = 0.f;
+        if (qi < len_q) {
+          const float lse = p.lse[row0 + qi];
+          l2v[e] = lse == -INFINITY ? -INFINITY : -lse * kLog2e;
+          drv[e] = p.drow[row0 + qi];
+        }
+      }
+      if (step >= NSTQ && !(ok = reduce_step(step - NSTQ))) break;
       if (lane == 0) {
         mbar_expect_tx(&s.q_full[st], 2 * Smem::kTileBytes);
 #pragma unroll
@@ -306,27 +344,23 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_4d(s.dout[st] + kb * BM * 128, &tm_do, &s.q_full[st], kb * 64, h, i0, b);
         }
       }
-      const long long row0 = ((long long)b * p.Hq + h) * p.Nq;
 #pragma unroll
       for (int e = 0; e < BM / 32; ++e) {
-        const int c = lane + 32 * e;
-        const int qi = i0 + c;
-        float l2 = -INFINITY, dr = 0.f;
-        if (qi < len_q) {
-          const float lse = p.lse[row0 + qi];
-          l2 = lse == -INFINITY ? -INFINITY : -lse * kLog2e;
-          dr = p.drow[row0 + qi];
-        }
-        s.nlse2[st][c] = l2;
-        s.drow[st][c] = dr;
+        s.nlse2[st][lane + 32 * e] = l2v[e];
+        s.drow[st][lane + 32 * e] = drv[e];
       }
       mbar_arrive(&s.q_full[st]);
       ++issued;
     }
-    if (lane == 0 && s.abort_flag) {
-      if (n_steps > 0) mbar_wait_drain(&s.kv_full, 0, p.wait_limit);
-      for (int j = max(0, issued - NSTQ); j < issued; ++j)
-        mbar_wait_drain(&s.q_full[j % NSTQ], (j / NSTQ) & 1, p.wait_limit);
+    // the last NSTQ dQ tiles
+    for (int t = max(0, n_steps - NSTQ); ok && t < n_steps; ++t) ok = reduce_step(t);
+    if (lane == 0) {
+      bulk_wait0();  // every reduction has completed before the CTA exits
+      if (s.abort_flag) {
+        if (n_steps > 0) mbar_wait_drain(&s.kv_full, 0, p.wait_limit);
+        for (int j = max(0, issued - NSTQ); j < issued; ++j)
+          mbar_wait_drain(&s.q_full[j % NSTQ], (j / NSTQ) & 1, p.wait_limit);
+      }
     }
   } else if (warp == 1) {
     // ===================================================== MMA issuer
@@ -339,20 +373,24 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int step = 0; ok && step < n_steps; ++step) {
         const int st = step % NSTQ;
         if (!mbar_wait(&s.q_full[st], (step / NSTQ) & 1, ab)) break;
-        // dP^T goes where dQ of the previous step was
-        if (step > 0 && !mbar_wait(&s.tmem_free, (step - 1) & 1, ab)) break;
         tc_fence_after();
         const uint32_t q_addr = smem_u32(s.q[st]), do_addr = smem_u32(s.dout[st]);
         // S^T = K_j Q_i^T (over P^T of the previous step, whose dV MMA was issued
         // earlier by this thread: tcgen05.mma executes in issue order) and
-        // dP^T = V_j dO_i^T, round-robin
+        // dP^T = V_j dO_i^T, round-robin.  dP^T goes where dQ of the previous
+        // step was: the first S^T MMA is issued before waiting for it to leave.
+        mma_ss(tmem + kColST, sdesc_sw128(k_addr, 16, 1024), sdesc_sw128(q_addr, 16, 1024), idesc_s, false);
+        if (step > 0 && !mbar_wait(&s.tmem_free, (step - 1) & 1, ab)) break;
+        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
-          mma_ss(tmem + kColST, sdesc_sw128(k_addr + off, 16, 1024), sdesc_sw128(q_addr + off, 16, 1024), idesc_s,
-                 kk > 0);
+          const uint32_t off1 = ((kk + 1) >> 2) * (128 * 128) + ((kk + 1) & 3) * 32;
           mma_ss(tmem + kColDPT, sdesc_sw128(v_addr + off, 16, 1024), sdesc_sw128(do_addr + off, 16, 1024),
                  idesc_s, kk > 0);
+          if (kk + 1 < D / 16)
+            mma_ss(tmem + kColST, sdesc_sw128(k_addr + off1, 16, 1024), sdesc_sw128(q_addr + off1, 16, 1024),
+                   idesc_s, true);
         }
         // its completion also implies that the previous step's MMAs, the last
         // readers of the dS^T tile, are done
@@ -377,9 +415,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit(&s.drain);
       mbar_wait_drain(&s.drain, 0, p.wait_limit);
     }
-  } else if (warp < 6) {
-    // ===================================================== P^T / dS^T (thread = key row)
-    const int quarter = warp & 3;
+  } else {
+    // ===================================================== elementwise groups
+    const int grp = (warp - 2) >> 2;  // 0: warps 2..5, 1: warps 6..9
+    const int quarter = warp & 3;     // TMEM lanes [32 quarter, 32 quarter + 32)
     const int r = quarter * 32 + lane;
     const int kj = n0 + r;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
@@ -404,31 +443,61 @@ __global__ void __launch_bounds__(kThreads, 1)
       if constexpr (BIAS == kBiasAlibi) neg_slope2 = -__ldg(p.alibi + h) * kLog2e;
       const uint32_t st_col = tmem + lane_off + kColST, dp_col = tmem + lane_off + kColDPT;
       if (need_mask)
-        bwd_p_chunks<true, BIAS>(st_col, s.nlse2[st], p.scale_log2, bcol, neg_slope2, p.Nk, i0, len_q, kj, len_k,
-                                 diag + p.win_r, p.win_l - diag, diag);
+        ok = bwd_p_half<true, BIAS>(grp, &s.s_read, step & 1, ab, st_col, s.nlse2[st], p.scale_log2, bcol,
+                                    neg_slope2, p.Nk, i0, len_q, kj, len_k, diag + p.win_r, p.win_l - diag, diag);
       else
-        bwd_p_chunks<false, BIAS>(st_col, s.nlse2[st], p.scale_log2, bcol, neg_slope2, p.Nk, i0, len_q, kj, len_k,
-                                  0, 0, diag);
+        ok = bwd_p_half<false, BIAS>(grp, &s.s_read, step & 1, ab, st_col, s.nlse2[st], p.scale_log2, bcol,
+                                     neg_slope2, p.Nk, i0, len_q, kj, len_k, 0, 0, diag);
+      if (!ok) break;
       tmem_wait_st();
-      bwd_ds_chunks(st_col, dp_col, s.drow[st], ds_row, r);
+      bwd_ds_half(grp, st_col, dp_col, s.drow[st], ds_row, r);
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s.ds_ready);
+      // ---- dQ_i (this thread: query row r, columns [grp D/2, grp D/2 + D/2))
+      ok = __all_sync(0xffffffffu, mbar_wait(&s.dkq_done, step & 1, ab));
+      if (!ok) break;
+      tc_fence_after();
+      uint32_t a[D / 2];
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c)
+        tmem_ld32(tmem + lane_off + kColDPT + grp * (D / 2) + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&a[c * 32]));
+      tmem_wait_ld();
+      reg_fence(a);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.tmem_free);
+      // box c (columns 32c .. 32c+31, 16 KB): each buffer holds D / 64 boxes,
+      // Q_i's first, then dO_i's; 128B-swizzled like the TMA map
+      const uint32_t q_row = smem_u32(s.q[st]) + r * 128, do_row = smem_u32(s.dout[st]) + r * 128;
+#pragma unroll
+      for (int cl = 0; cl < D / 64; ++cl) {
+        const int c = grp * (D / 64) + cl;
+        const uint32_t row = (c < kBoxes ? q_row : do_row) + (c % kBoxes) * (128 * 128);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int e = cl * 32 + 4 * u;
+          st_shared_v4(row + ((u ^ (r & 7)) << 4), a[e], a[e + 1], a[e + 2], a[e + 3]);
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.staged[st]);
     }
-    // ---- epilogue: dK (scaled) and dV for this thread's key row
+    // ---- epilogue: dK (scaled) and dV, key row r, columns [grp D/2, grp D/2 + D/2)
     // the MMA warp commits `drain` after its last MMA
     if (ok && n_steps > 0) ok = __all_sync(0xffffffffu, mbar_wait(&s.drain, 0, ab));
     tc_fence_after();
     if (ok) {
-      const long long row = (((long long)b * p.Nk + kj) * p.Hkv + hk) * D;
+      const long long row = (((long long)b * p.Nk + kj) * p.Hkv + hk) * D + grp * (D / 2);
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
-        const uint32_t col0 = half == 0 ? kColDV : kColDK;
+        const uint32_t col0 = (half == 0 ? kColDV : kColDK) + grp * (D / 2);
         const float mul = half == 0 ? 1.f : p.scale;
         __nv_bfloat16* dst = (half == 0 ? p.dv : p.dk) + row;
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c) {
+        for (int c = 0; c < D / 64; ++c) {
           uint32_t a[32];
           if (n_steps > 0) {
             tmem_ld32(tmem + lane_off + col0 + c * 32, a);
@@ -450,58 +519,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
-  } else {
-    // ===================================================== dQ drain (thread = query row)
-    // dQ_i is read out of TMEM at once (freeing its columns for the next dP^T),
-    // staged through the step's own Q_i / dO_i buffers -- four 128-row x 32-column
-    // fp32 boxes, 128B-swizzled like the TMA map -- and added to the fp32
-    // accumulator by TMA bulk reductions; the producer refills the buffers once
-    // the reductions have read them.
-    const int quarter = warp & 3;
-    const int r = quarter * 32 + lane;
-    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const bool leader = warp == 6 && lane == 0;
-    for (int step = 0; step < n_steps; ++step) {
-      const int st = step % NSTQ;
-      const int h = hk * G + step / per_head;
-      const int i0 = (i_first + step % per_head) * BM;
-      // every MMA of the step is done: dQ_i is final and Q_i / dO_i are unused
-      if (!__all_sync(0xffffffffu, mbar_wait(&s.dkq_done, step & 1, ab))) break;
-      tc_fence_after();
-      uint32_t a[D];
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) tmem_ld32(tmem + lane_off + kColDPT + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&a[c * 32]));
-      tmem_wait_ld();
-      reg_fence(a);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s.tmem_free);
-      // box c (columns 32c .. 32c+31, 16 KB): each buffer holds D / 64 boxes,
-      // Q_i's first, then dO_i's
-      constexpr int kBoxes = D / 64;
-      const uint32_t q_row = smem_u32(s.q[st]) + r * 128, do_row = smem_u32(s.dout[st]) + r * 128;
-#pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
-        const uint32_t row = (c < kBoxes ? q_row : do_row) + (c % kBoxes) * (128 * 128);
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int e = c * 32 + 4 * u;
-          st_shared_v4(row + ((u ^ (r & 7)) << 4), a[e], a[e + 1], a[e + 2], a[e + 3]);
-        }
-      }
-      fence_proxy_async_smem();
-      named_bar_sync(1, 128);
-      if (leader) {
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c)
-          tma_reduce_add_4d(&tm_dq, (c < kBoxes ? s.q[st] : s.dout[st]) + (c % kBoxes) * (128 * 128), c * 32, h, i0, b);
-        bulk_commit();
-        bulk_wait_read0();
-        mbar_arrive(&s.q_free[st]);
-      }
-      __syncwarp();
-    }
-    if (leader) bulk_wait0();
   }
 
   tc_fence_before();
