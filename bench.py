@@ -50,7 +50,7 @@ def parse_args(argv=None):
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip timing the CPU oracle")
-    ap.add_argument("--workload", default="c3", choices=["c1", "c2", "c3", "c4", "c5a", "c5b"],
+    ap.add_argument("--workload", default="c3", choices=["c1", "c2", "c3", "c4", "c5a", "c5b", "kv1"],
                     help="c3 (default) is the headline causal fwd+bwd workload; the others are reported too")
     ap.add_argument("--batch", type=int, default=None, help="override the batch (profiling a smaller case)")
     ap.add_argument("--heads", type=int, default=None, help="override the head count (profiling a smaller case)")
@@ -58,6 +58,8 @@ def parse_args(argv=None):
                     help="grouped workload: read the dense fp32 bias tensor, or form it in-kernel from slopes")
     ap.add_argument("--window", type=int, default=None,
                     help="causal sliding window: each row sees its own and at most WINDOW earlier keys")
+    ap.add_argument("--num-splits", type=int, default=0,
+                    help="split-KV workload: key splits (0: the library's choice, 1: a single pass)")
     ap.add_argument("--naive", action="store_true",
                     help="time the fused forward against the materialising three-kernel comparator instead")
     return ap.parse_args(argv)
@@ -260,7 +262,8 @@ def make_job(w, args, dev, rank):
             attn.attn_fwd_varlen(j.dev["q"], j.dev["k"], j.dev["v"], cu, cu, mx, mx, causal=w.causal,
                                  out=j.out["o"], lse=j.out["lse"])
     else:
-        inp = synth.make_dense(w.batch, w.h_q, w.h_kv, w.n, w.n, w.d, dtype=dtype, sigma_qk=w.sigma_qk, seed=seed,
+        n_q = w.n_q or w.n
+        inp = synth.make_dense(w.batch, w.h_q, w.h_kv, n_q, w.n, w.d, dtype=dtype, sigma_qk=w.sigma_qk, seed=seed,
                                with_dout=w.backward)
         names = ("q", "k", "v", "dout") if w.backward else ("q", "k", "v")
         j.host = {n: getattr(inp, n).pin_memory() for n in names}
@@ -270,7 +273,7 @@ def make_job(w, args, dev, rank):
             # the same bias from its per-head slopes, formed inside the kernels
             j.host["alibi"] = synth.alibi_like_slopes(w.h_q).pin_memory()
         j.dev = {n: t.to(dev) for n, t in j.host.items()}
-        j.out = {"o": torch.empty_like(j.dev["q"]), "lse": torch.empty((w.batch, w.h_q, w.n), device=dev)}
+        j.out = {"o": torch.empty_like(j.dev["q"]), "lse": torch.empty((w.batch, w.h_q, n_q), device=dev)}
         win = None if args.window is None else (int(args.window), None)
         ws = None
         if w.backward:
@@ -278,8 +281,18 @@ def make_job(w, args, dev, rank):
                          dv=torch.empty_like(j.dev["v"]))
             ws = torch.empty(attn.attn_bwd_workspace_size(w.batch, w.h_q, w.n, w.d), device=dev, dtype=torch.uint8)
 
+        if w.splitkv:
+            t = args.num_splits or attn.attn_splitkv_num_splits(w.batch, w.h_q, n_q, w.n)
+            j.splits = t
+            sws = torch.empty(max(256, attn._lib.attn_splitkv_workspace_size(w.batch, w.h_q, n_q, w.d, t)),
+                              device=dev, dtype=torch.uint8)
+
         def step():
             d_, o_ = j.dev, j.out
+            if w.splitkv:
+                attn.attn_fwd_splitkv(d_["q"], d_["k"], d_["v"], causal=w.causal, num_splits=j.splits, out=o_["o"],
+                                      lse=o_["lse"], workspace=sws)
+                return
             attn.attn_fwd(d_["q"], d_["k"], d_["v"], bias=d_.get("bias"), causal=w.causal, out=o_["o"], lse=o_["lse"],
                           alibi_slopes=d_.get("alibi"), window=win)
             if w.backward:
@@ -425,6 +438,7 @@ def run_ours(args):
             "data": f"synthetic (seeded randn; Q/K std {w.sigma_qk:g}, V/dO std 1)",
             "config": {"workload": w.name, "batch": w.batch, "heads": w.h_q, "kv_heads": w.h_kv,
                        "seq_len": w.n if not w.varlen else f"{w.num_seqs} seqs, {int(sum(job.lengths))} tokens",
+                       **({"query_len": w.n_q, "num_splits": job.splits} if w.splitkv else {}),
                        "head_dim": w.d, "causal": w.causal,
                        "bias": (("dense fp32 tensor" if args.bias_mode == "dense" else "per-head slopes, formed in-kernel")
                                 if w.bias else False), "backward": w.backward,

@@ -38,6 +38,10 @@ EXPORTS = {
     "attn_fwd_local": (_I, [_VP, _VP, _VP, _FP, _VP, _FP, _I, _I, _I, _I, _I, _I, _F, _I, _I, _I, _I, _VP]),
     "attn_bwd_local": (_I, [_VP, _VP, _VP, _FP, _VP, _FP, _VP, _VP, _VP, _VP, _VP, _SZ, _I, _I, _I, _I, _I, _I,
                             _F, _I, _I, _I, _I, _VP]),
+    "attn_splitkv_num_splits": (_I, [_I, _I, _I, _I]),
+    "attn_splitkv_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
+    "attn_fwd_splitkv": (_I, [_VP, _VP, _VP, _VP, _FP, _I, _I, _I, _I, _I, _I, _F, _I, _I, _VP, _SZ, _I, _VP]),
+    "attn_merge_partials": (_I, [_FP, _FP, _I, _VP, _FP, _I, _I, _I, _I, _I, _VP]),
     "attn_bwd_workspace_size": (_SZ, [_I, _I, _I, _I]),
     "attn_bwd": (_I, [_VP, _VP, _VP, _FP, _LL, _VP, _FP, _VP, _VP, _VP, _VP, _VP, _SZ, _I, _I, _I, _I, _I,
                       _I, _F, _I, _I, _VP]),
@@ -160,6 +164,43 @@ def attn_fwd(q, k, v, bias=None, causal=False, scale=None, out=None, lse=None, s
     bp, bs = _bias_args(bias, B, Hq, Nq, Nk)
     _check(_lib.attn_fwd(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), bp, bs, _dev(o, "o"), _dev(lse, "lse"),
                          B, Hq, Hkv, Nq, Nk, d, scale, int(bool(causal)), _dtype_code(q), _stream(stream)))
+    return o, lse
+
+
+def attn_splitkv_num_splits(batch, h_q, n_q, n_k) -> int:
+    return int(_lib.attn_splitkv_num_splits(batch, h_q, n_q, n_k))
+
+
+def attn_fwd_splitkv(q, k, v, causal=False, scale=None, num_splits=0, out=None, lse=None, workspace=None,
+                     stream=None):
+    """attn_fwd computed over num_splits key ranges and merged (bf16, dense)."""
+    B, Nq, Hq, d = q.shape
+    Nk, Hkv = k.shape[1], k.shape[2]
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    o = torch.empty_like(q) if out is None else out
+    lse = torch.empty((B, Hq, Nq), device=q.device, dtype=torch.float32) if lse is None else lse
+    t = int(num_splits) if num_splits and num_splits > 0 else attn_splitkv_num_splits(B, Hq, Nq, Nk)
+    if workspace is None:
+        workspace = torch.empty(max(256, int(_lib.attn_splitkv_workspace_size(B, Hq, Nq, d, t))), device=q.device,
+                                dtype=torch.uint8)
+    _check(_lib.attn_fwd_splitkv(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(o, "o"), _dev(lse, "lse"), B, Hq,
+                                 Hkv, Nq, Nk, d, scale, int(bool(causal)), t, _dev(workspace, "workspace"),
+                                 workspace.numel() * workspace.element_size(), _dtype_code(q), _stream(stream)))
+    return o, lse
+
+
+def attn_merge_partials(o_parts, lse_parts, out=None, lse=None, out_dtype=torch.bfloat16, stream=None):
+    """Merge fp32 partials o_parts [T,B,Nq,Hq,d], lse_parts [T,B,Hq,Nq] over disjoint key ranges."""
+    if o_parts.dtype != torch.float32 or lse_parts.dtype != torch.float32:
+        raise AttnError("partials must be fp32")
+    T, B, Nq, Hq, d = o_parts.shape
+    o = torch.empty((B, Nq, Hq, d), device=o_parts.device, dtype=out_dtype) if out is None else out
+    lse = torch.empty((B, Hq, Nq), device=o_parts.device, dtype=torch.float32) if lse is None else lse
+    code = 0 if o.dtype == torch.bfloat16 else 1 if o.dtype == torch.float32 else None
+    if code is None:
+        raise AttnError("merge output must be bf16 or fp32")
+    _check(_lib.attn_merge_partials(_dev(o_parts, "o_parts"), _dev(lse_parts, "lse_parts"), T, _dev(o, "o"),
+                                    _dev(lse, "lse"), B, Hq, Nq, d, code, _stream(stream)))
     return o, lse
 
 

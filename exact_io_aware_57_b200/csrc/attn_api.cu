@@ -2,6 +2,8 @@
 // validation, dispatch by dtype / head dim / bias, workspace carving, and the
 // device status word.  Nothing here computes attention; every step of the
 // path runs in the kernels.
+#include <algorithm>
+
 #include <mutex>
 
 #include "common.cuh"
@@ -290,6 +292,83 @@ int attn_bwd_local(const void* q, const void* k, const void* v, const float* ali
                    int causal, int window_left, int window_right, int dtype, void* stream) {
   return bwd_impl(q, k, v, nullptr, 0, alibi_slopes, o, lse, dout, dq, dk, dv, workspace, workspace_bytes, batch,
                   h_q, h_kv, n_q, n_k, d, scale, causal, window_left, window_right, dtype, stream);
+}
+
+int attn_splitkv_num_splits(int batch, int h_q, int n_q, int n_k) {
+  if (batch <= 0 || h_q <= 0 || n_q <= 0 || n_k <= 0) return 1;
+  const long long ctas = (long long)((n_q + 127) / 128) * h_q * batch;
+  const int kv_tiles = (n_k + 127) / 128;
+  // One CTA per SM at a time (the forward holds all of TMEM): pick the split
+  // count whose last wave is fullest, preferring fewer splits (each adds a
+  // merge pass and a pipeline start); splits keep at least four key tiles.
+  const int t_max = (int)std::max(1, std::min(64, kv_tiles / 4));
+  auto fill = [&](long long t) {
+    const long long n = ctas * t;
+    return (double)n / (double)(((n + 147) / 148) * 148);
+  };
+  int best = 1;
+  for (int t = 2; t <= t_max; ++t)
+    if (fill(t) > fill(best) + 0.05) best = t;
+  return best;
+}
+
+size_t attn_splitkv_workspace_size(int batch, int h_q, int n_q, int d, int num_splits) {
+  if (batch <= 0 || h_q <= 0 || n_q <= 0 || d <= 0 || num_splits <= 0) return 0;
+  const size_t rows = (size_t)batch * n_q * h_q;
+  return align256(rows * d * num_splits * sizeof(float)) + align256(rows * num_splits * sizeof(float));
+}
+
+int attn_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse, int batch, int h_q, int h_kv,
+                     int n_q, int n_k, int d, float scale, int causal, int num_splits, void* workspace,
+                     size_t workspace_bytes, int dtype, void* stream) {
+  int rc = check_common(batch, h_q, h_kv, n_q, n_k, d, dtype);
+  if (rc) return rc;
+  if (dtype != ATTN_BF16) return ATTN_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return ATTN_ERR_INVALID;
+  if (!supported_device()) return ATTN_ERR_UNSUPPORTED;
+  if (num_splits <= 0) num_splits = attn_splitkv_num_splits(batch, h_q, n_q, n_k);
+  const int kv_tiles = (n_k + 127) / 128;
+  const int tiles_per_split = (kv_tiles + std::min(num_splits, kv_tiles) - 1) / std::min(num_splits, kv_tiles);
+  const int splits = (kv_tiles + tiles_per_split - 1) / tiles_per_split;  // none of them empty
+  TcGeom g{};
+  g.q = q;
+  g.k = k;
+  g.v = v;
+  g.B = batch;
+  g.Hq = h_q;
+  g.Hkv = h_kv;
+  g.Nq = n_q;
+  g.Nk = n_k;
+  g.D = d;
+  g.causal = causal != 0;
+  g.scale = scale;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (splits == 1) return launch_fwd_sm100(g, static_cast<__nv_bfloat16*>(o), lse, st);
+  const size_t need = attn_splitkv_workspace_size(batch, h_q, n_q, d, splits);
+  if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return ATTN_ERR_WORKSPACE;
+  const size_t rows = (size_t)batch * n_q * h_q;
+  SplitKV sp;
+  sp.num_splits = splits;
+  sp.split_len = tiles_per_split * 128;
+  sp.o_part = static_cast<float*>(workspace);
+  sp.lse_part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + align256(rows * d * splits * sizeof(float)));
+  rc = launch_fwd_sm100(g, static_cast<__nv_bfloat16*>(o), lse, st, &sp);
+  if (rc) return rc;
+  return launch_merge(sp.o_part, sp.lse_part, splits, o, lse, batch, h_q, n_q, d, 0, st);
+}
+
+int attn_merge_partials(const float* o_parts, const float* lse_parts, int num_parts, void* o, float* lse, int batch,
+                        int h_q, int n_q, int d, int out_dtype, void* stream) {
+  if (!o_parts || !lse_parts || !o || !lse || num_parts <= 0 || batch <= 0 || h_q <= 0 || n_q <= 0)
+    return ATTN_ERR_INVALID;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if (out_dtype != ATTN_BF16 && out_dtype != ATTN_F32) return ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(o_parts) || !aligned16(o)) return ATTN_ERR_INVALID;
+  if (!supported_device()) return ATTN_ERR_UNSUPPORTED;
+  return launch_merge(o_parts, lse_parts, num_parts, o, lse, batch, h_q, n_q, d, out_dtype == ATTN_F32,
+                      static_cast<cudaStream_t>(stream));
 }
 
 int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse, const int* cu_seqlens_q,

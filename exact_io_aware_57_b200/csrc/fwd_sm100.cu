@@ -27,6 +27,12 @@
 // key visible from some row of the tile are loaded ("Understanding
 // FlashAttention Pt 1", contents 3.5 tile skipping and 4.2 local attention);
 // the mask is applied only on tiles that straddle the visible band.
+// Split-KV: with num_splits > 1 the grid's z index also runs over splits of
+// the keys (split_len keys each, a multiple of the tile); every CTA then
+// writes its exact partial result -- O_t normalised in fp32 and LSE_t -- and a
+// separate merge combines the splits with weights exp(LSE_t - LSE), the
+// rescale-and-add of "Softmax does not need the matrix", "Carry the
+// Normalizer", applied to whole splits.
 #include <algorithm>
 
 #include "common.cuh"
@@ -74,6 +80,10 @@ struct FwdParams {
   float scale_log2;
   int causal;
   int win_l, win_r;  // key j visible from row i iff i + diag - win_l <= j <= i + diag + win_r
+  int num_splits, split_len;           // split-KV (1, unused: one split)
+  float* o_part;                       // [num_splits, B, Nq, Hq, D] fp32, or null: O in bf16 to o
+  float* lse_part;                     // [num_splits, B, Hq, Nq]
+  long long part_o_stride, part_lse_stride;
   int* status;
   long long wait_limit;
 };
@@ -85,7 +95,7 @@ ATTN_DEVINL void reg_fence(uint32_t (&r)[N]) {
   for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
 }
 
-template <int D, int BIAS, bool FAST>
+template <int D, int BIAS, bool FAST, bool PARTIAL>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
@@ -99,7 +109,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // ---- work tile: heavy (late) query tiles first under causal masking
   const int m_tile = p.causal ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x;
-  const int h = blockIdx.y, z = blockIdx.z;
+  const int h = blockIdx.y;
+  const int z = PARTIAL ? (int)blockIdx.z / p.num_splits : (int)blockIdx.z;
+  const int split = PARTIAL ? (int)blockIdx.z % p.num_splits : 0;
   int q_off = 0, len_q = p.Nq, k_off = 0, len_k = p.Nk, bidx = z;
   if (p.cu_q) {
     q_off = p.cu_q[z];
@@ -113,8 +125,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int hk = h / (p.Hq / p.Hkv);
   const int diag = len_k - len_q;  // row i is aligned with key i + diag
   // keys [kv_begin, kv_end) hold every key visible from rows m0 .. m0 + BM - 1
-  const int kv_end = min(len_k, m0 + BM + diag + p.win_r);
-  const int kv_begin = max(0, m0 + diag - p.win_l);
+  // ... clipped to this CTA's split of the keys
+  const int kv_end = min(PARTIAL ? min(len_k, (split + 1) * p.split_len) : len_k, m0 + BM + diag + p.win_r);
+  const int kv_begin = max(PARTIAL ? split * p.split_len : 0, m0 + diag - p.win_l);
   const int j_first = kv_begin / BN;
   const int n_kv = kv_end > kv_begin ? (kv_end + BN - 1) / BN - j_first : 0;
 
@@ -348,6 +361,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok) {
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
       __nv_bfloat16* orow = p.o + bidx * p.o_bstride + ((long long)(q_off + i) * p.Hq + h) * D;
+      float* prow = nullptr;
+      if constexpr (PARTIAL) prow = p.o_part + split * p.part_o_stride + bidx * p.o_bstride +
+                                    ((long long)(q_off + i) * p.Hq + h) * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         uint32_t orr[32];
@@ -358,6 +374,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
 #pragma unroll
           for (int e = 0; e < 32; ++e) orr[e] = 0u;
+        }
+        if constexpr (PARTIAL) {  // split partial: fp32
+          if (row_ok) {
+            float4* dst = reinterpret_cast<float4*>(prow + c * 32);
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              dst[e] = make_float4(__uint_as_float(orr[4 * e]) * inv_l, __uint_as_float(orr[4 * e + 1]) * inv_l,
+                                   __uint_as_float(orr[4 * e + 2]) * inv_l, __uint_as_float(orr[4 * e + 3]) * inv_l);
+          }
+          continue;
         }
         uint32_t packed[16];
 #pragma unroll
@@ -370,9 +396,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             dst[e] = make_uint4(packed[4 * e], packed[4 * e + 1], packed[4 * e + 2], packed[4 * e + 3]);
         }
       }
-      if (row_ok)
-        p.lse[bidx * p.lse_bstride + (long long)h * p.lse_hstride + q_off + i] =
-            l > 0.f ? (m + __log2f(l)) * kLn2 : -INFINITY;
+      if (row_ok) {
+        const float lse = l > 0.f ? (m + __log2f(l)) * kLn2 : -INFINITY;
+        if constexpr (PARTIAL)
+          p.lse_part[split * p.part_lse_stride + bidx * p.lse_bstride + (long long)h * p.lse_hstride + q_off + i] = lse;
+        else
+          p.lse[bidx * p.lse_bstride + (long long)h * p.lse_hstride + q_off + i] = lse;
+      }
     }
   }
 
@@ -386,17 +416,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D, int BIAS, bool FAST>
+template <int D, int BIAS, bool FAST, bool PARTIAL = false>
 int launch_fwd_t(const TcGeom& g, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                  const FwdParams& p, cudaStream_t st) {
   // At least half of the SM's shared memory, so that a second CTA never waits
   // on the 512 TMEM columns this one holds.
   const size_t smem = std::max<size_t>(sizeof(FwdSmem<D>) + 1024, 116 * 1024);
-  auto kern = fwd_sm100_kernel<D, BIAS, FAST>;
+  auto kern = fwd_sm100_kernel<D, BIAS, FAST, PARTIAL>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return ATTN_ERR_CUDA;
   const int max_nq = g.cu_q ? g.max_nq : g.Nq;
-  dim3 grid((max_nq + BM - 1) / BM, g.Hq, g.cu_q ? g.num_seqs : g.B);
+  dim3 grid((max_nq + BM - 1) / BM, g.Hq, (g.cu_q ? g.num_seqs : g.B) * p.num_splits);
   record_kernel_event(ATTN_KERNEL_FWD, 0, st);
   kern<<<grid, kThreads, smem, st>>>(mq, mk, mv, p);
   record_kernel_event(ATTN_KERNEL_FWD, 1, st);
@@ -406,7 +436,7 @@ int launch_fwd_t(const TcGeom& g, const CUtensorMap& mq, const CUtensorMap& mk, 
 
 }  // namespace
 
-int launch_fwd_sm100(const TcGeom& g, __nv_bfloat16* o, float* lse, cudaStream_t st) {
+int launch_fwd_sm100(const TcGeom& g, __nv_bfloat16* o, float* lse, cudaStream_t st, const SplitKV* split) {
   // 4-D views (d, head, row, batch); packed inputs are one batch of `total` rows.
   const int B = g.cu_q ? 1 : g.B;
   CUtensorMap mq, mk, mv;
@@ -441,11 +471,28 @@ int launch_fwd_sm100(const TcGeom& g, __nv_bfloat16* o, float* lse, cudaStream_t
   p.causal = g.causal;
   p.win_l = win_left(g.window_left);
   p.win_r = win_right(g.causal, g.window_right);
+  p.num_splits = 1;
+  p.split_len = g.Nk;
+  if (split) {  // dense inputs only
+    p.num_splits = split->num_splits;
+    p.split_len = split->split_len;
+    p.o_part = split->o_part;
+    p.lse_part = split->lse_part;
+    p.part_o_stride = (long long)g.B * g.Nq * g.Hq * g.D;
+    p.part_lse_stride = (long long)g.B * g.Hq * g.Nq;
+  }
   p.status = device_status_ptr();
   p.wait_limit = kWaitLimitCycles;
   if (!p.status) return ATTN_ERR_CUDA;
   // FAST: no bias and a positive scale, so the row max can be taken on raw scores
   const bool fast = !g.bias && !g.alibi && g.scale > 0.f;
+  if (split) {  // no bias on this path
+    if (g.D == 64)
+      return fast ? launch_fwd_t<64, kBiasNone, true, true>(g, mq, mk, mv, p, st)
+                  : launch_fwd_t<64, kBiasNone, false, true>(g, mq, mk, mv, p, st);
+    return fast ? launch_fwd_t<128, kBiasNone, true, true>(g, mq, mk, mv, p, st)
+                : launch_fwd_t<128, kBiasNone, false, true>(g, mq, mk, mv, p, st);
+  }
   if (g.D == 64) {
     if (g.bias) return launch_fwd_t<64, kBiasDense, false>(g, mq, mk, mv, p, st);
     if (g.alibi) return launch_fwd_t<64, kBiasAlibi, false>(g, mq, mk, mv, p, st);

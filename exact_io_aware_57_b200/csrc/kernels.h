@@ -71,7 +71,18 @@ struct TcGeom {
   int window_left = -1, window_right = -1;  // local attention sizes; negative: unbounded
 };
 
-int launch_fwd_sm100(const TcGeom& g, __nv_bfloat16* o, float* lse, cudaStream_t st);
+// Split-KV forward: keys cut into num_splits ranges of split_len (a multiple of
+// 128); each writes O_t (fp32, normalised) and LSE_t for the merge.
+struct SplitKV {
+  int num_splits, split_len;
+  float* o_part;    // [num_splits, B, Nq, Hq, D]
+  float* lse_part;  // [num_splits, B, Hq, Nq]
+};
+int launch_fwd_sm100(const TcGeom& g, __nv_bfloat16* o, float* lse, cudaStream_t st, const SplitKV* split = nullptr);
+// O = sum_t exp(LSE_t - LSE) O_t, LSE = log sum_t exp(LSE_t) over num_parts
+// partials laid out as SplitKV's; o: bf16 (out_f32 = 0) or fp32 [B, Nq, Hq, D].
+int launch_merge(const float* o_part, const float* lse_part, int num_parts, void* o, float* lse, int B, int Hq,
+                 int Nq, int D, int out_f32, cudaStream_t st);
 int launch_bwd_sm100(const TcGeom& g, const __nv_bfloat16* o, const float* lse, const __nv_bfloat16* dout,
                      __nv_bfloat16* dq, __nv_bfloat16* dk, __nv_bfloat16* dv, float* dq_acc, float* Drow,
                      cudaStream_t st);

@@ -30,6 +30,8 @@ class Workload:
     num_seqs: int = 0
     len_lo: int = 0
     len_hi: int = 0
+    n_q: int = 0              # query length when it differs from n (the key length)
+    splitkv: bool = False     # forward through the split-KV path
     description: str = field(default="", compare=False)
 
 
@@ -47,6 +49,10 @@ WORKLOADS = {
     "c5a": Workload("varlen causal bf16 16 seqs L~U[512,8192] H=32 d=128 fwd", 1, 32, 32, 0, 128, "bf16",
                     True, False, varlen=True, num_seqs=16, len_lo=512, len_hi=8192,
                     description="16 packed sequences, lengths uniform in [512, 8192] from the seed"),
+    "kv1": Workload("split-KV: causal bf16 B=1 Hq=32 Hkv=8 Nq=512 Nk=65536 d=128 fwd", 1, 32, 8, 65536, 128,
+                    "bf16", True, False, n_q=512, splitkv=True,
+                    description="a 512-query block at the end of a 65536-key sequence (bottom-right causal), "
+                                "GQA 32:8: 128 query-tile CTAs alone would not fill 148 SMs"),
     "c5b": Workload("single sequence causal bf16 N=32768 H=16 d=128 fwd", 1, 16, 16, 32768, 128, "bf16",
                     True, False,
                     description="one sequence of 32768 tokens, 16 heads, causal, forward"),
@@ -71,6 +77,10 @@ def flops(w: Workload, backward: bool | None = None, lengths=None, window: int |
     causal sliding ``window`` (keys i - window .. i) the count is 4*d per
     visible pair, pairs counted exactly."""
     bwd = w.backward if backward is None else backward
+    if w.n_q:
+        nq, nk = w.n_q, w.n
+        pairs = nq * (nk - nq) + nq * (nq + 1) // 2 if w.causal else nq * nk
+        return 4.0 * w.d * pairs * w.batch * w.h_q * (3.5 if bwd else 1.0)
     if window is not None:
         assert not w.varlen and w.causal
         f = 4.0 * w.d * window_pairs(w.n, window) * w.batch * w.h_q

@@ -127,6 +127,41 @@ int attn_bwd_local(const void* q, const void* k, const void* v, const float* ali
                    int dtype, void* stream);
 
 /*
+ * Split-KV forward: the keys are cut into num_splits contiguous ranges (whole
+ * 128-key tiles); each (query tile, head, batch, split) is an independent CTA
+ * that writes the exact attention of its rows over its own keys (O_t fp32,
+ * LSE_t) to the workspace, and attn_merge_partials' kernel combines them into
+ * o (bf16) and lse.  The result is the same function as attn_fwd; it gives a
+ * launch enough CTAs when batch x heads x query tiles is small against the
+ * 148 SMs (short query blocks over long key sequences).  num_splits <= 0
+ * takes attn_splitkv_num_splits' choice; splits that would be empty are
+ * dropped.  bf16 only (ATTN_ERR_UNSUPPORTED for fp32); dense inputs, no bias.
+ * workspace: DEVICE, 256-byte aligned, attn_splitkv_workspace_size(batch, h_q,
+ * n_q, d, num_splits) bytes (not needed when one split results).
+ */
+int attn_splitkv_num_splits(int batch, int h_q, int n_q, int n_k);
+size_t attn_splitkv_workspace_size(int batch, int h_q, int n_q, int d, int num_splits);
+int attn_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse, int batch,
+                     int h_q, int h_kv, int n_q, int n_k, int d, float scale, int causal,
+                     int num_splits, void* workspace, size_t workspace_bytes, int dtype,
+                     void* stream);
+
+/*
+ * Merge exact partial results over disjoint key ranges (split-KV, or keys
+ * sharded across devices and gathered): with m = max_t LSE_t and
+ * w_t = exp(LSE_t - m), O = sum_t w_t O_t / sum_t w_t and
+ * LSE = m + ln sum_t w_t; rows whose LSE_t are all -inf get O = 0, LSE = -inf
+ * ("Softmax does not need the matrix", "Carry the Normalizer": the carried
+ * running state resumes the softmax exactly).
+ * o_parts: DEVICE fp32 [num_parts, batch, n_q, h_q, d] (each O_t normalised);
+ * lse_parts: DEVICE fp32 [num_parts, batch, h_q, n_q]; o: DEVICE
+ * [batch, n_q, h_q, d] of out_dtype (ATTN_BF16 or ATTN_F32); lse: DEVICE fp32
+ * [batch, h_q, n_q].  d in {64, 128}.
+ */
+int attn_merge_partials(const float* o_parts, const float* lse_parts, int num_parts, void* o,
+                        float* lse, int batch, int h_q, int n_q, int d, int out_dtype, void* stream);
+
+/*
  * attn_bwd without a workspace argument, for callers that cannot allocate
  * device memory when they run the backward (code inside a framework that owns
  * all device memory, or latency-critical loops that cannot afford cudaMalloc's
