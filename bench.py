@@ -58,6 +58,8 @@ def parse_args(argv=None):
                     help="grouped workload: read the dense fp32 bias tensor, or form it in-kernel from slopes")
     ap.add_argument("--window", type=int, default=None,
                     help="causal sliding window: each row sees its own and at most WINDOW earlier keys")
+    ap.add_argument("--with-backward", action="store_true",
+                    help="packed workload: time the forward and the backward (attn_bwd_varlen)")
     ap.add_argument("--num-splits", type=int, default=0,
                     help="split-KV workload: key splits (0: the library's choice, 1: a single pass)")
     ap.add_argument("--naive", action="store_true",
@@ -251,16 +253,26 @@ def make_job(w, args, dev, rank):
     j = types.SimpleNamespace(w=w, lengths=None)
     if w.varlen:
         j.lengths = synth.varlen_lengths(w.num_seqs, w.len_lo, w.len_hi, seed=args.seed)
-        inp = synth.make_packed(j.lengths, w.h_q, w.h_kv, w.d, dtype=dtype, seed=seed)
-        j.host = {"q": inp.q.pin_memory(), "k": inp.k.pin_memory(), "v": inp.v.pin_memory()}
+        inp = synth.make_packed(j.lengths, w.h_q, w.h_kv, w.d, dtype=dtype, seed=seed, with_dout=w.backward)
+        names = ("q", "k", "v", "dout") if w.backward else ("q", "k", "v")
+        j.host = {n: getattr(inp, n).pin_memory() for n in names}
         j.dev = {n: t.to(dev) for n, t in j.host.items()}
         cu = inp.cu_seqlens.to(dev)
         mx = int(max(j.lengths))
         j.out = {"o": torch.empty_like(j.dev["q"]), "lse": torch.empty((w.h_q, inp.q.shape[0]), device=dev)}
+        if w.backward:
+            j.out.update(dq=torch.empty_like(j.dev["q"]), dk=torch.empty_like(j.dev["k"]),
+                         dv=torch.empty_like(j.dev["v"]))
+            vws = torch.empty(attn.attn_bwd_workspace_size(1, w.h_q, inp.q.shape[0], w.d), device=dev,
+                              dtype=torch.uint8)
 
         def step():
             attn.attn_fwd_varlen(j.dev["q"], j.dev["k"], j.dev["v"], cu, cu, mx, mx, causal=w.causal,
                                  out=j.out["o"], lse=j.out["lse"])
+            if w.backward:
+                attn.attn_bwd_varlen(j.dev["q"], j.dev["k"], j.dev["v"], j.out["o"], j.out["lse"], j.dev["dout"],
+                                     cu, cu, mx, mx, causal=w.causal, workspace=vws, dq=j.out["dq"],
+                                     dk=j.out["dk"], dv=j.out["dv"])
     else:
         n_q = w.n_q or w.n
         inp = synth.make_dense(w.batch, w.h_q, w.h_kv, n_q, w.n, w.d, dtype=dtype, sigma_qk=w.sigma_qk, seed=seed,
@@ -328,6 +340,8 @@ def run_ours(args):
     dev = torch.device("cuda", local)
     dist = init_dist(world, "nccl")
     w = workloads.WORKLOADS[args.workload]
+    if args.with_backward and w.varlen and not w.backward:
+        w = dataclasses.replace(w, name=w.name.replace(" fwd", " fwd+bwd"), backward=True)
     if args.batch or args.heads:
         w = dataclasses.replace(w, name=w.name + " (reduced for profiling)", batch=args.batch or w.batch,
                                 h_q=args.heads or w.h_q, h_kv=args.heads or w.h_kv)

@@ -38,6 +38,8 @@ EXPORTS = {
     "attn_fwd_local": (_I, [_VP, _VP, _VP, _FP, _VP, _FP, _I, _I, _I, _I, _I, _I, _F, _I, _I, _I, _I, _VP]),
     "attn_bwd_local": (_I, [_VP, _VP, _VP, _FP, _VP, _FP, _VP, _VP, _VP, _VP, _VP, _SZ, _I, _I, _I, _I, _I, _I,
                             _F, _I, _I, _I, _I, _VP]),
+    "attn_bwd_varlen": (_I, [_VP, _VP, _VP, _VP, _FP, _VP, _VP, _VP, _VP, _IP, _IP, _I, _I, _I, _I, _I, _I, _I, _I,
+                             _F, _I, _VP, _SZ, _I, _VP]),
     "attn_splitkv_num_splits": (_I, [_I, _I, _I, _I]),
     "attn_splitkv_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
     "attn_fwd_splitkv": (_I, [_VP, _VP, _VP, _VP, _FP, _I, _I, _I, _I, _I, _I, _F, _I, _I, _VP, _SZ, _I, _VP]),
@@ -261,6 +263,28 @@ def attn_fwd_varlen(q, k, v, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqle
                                 cu_seqlens_q.numel() - 1, int(max_seqlen_q), int(max_seqlen_k), Tq, Tk, Hq, Hkv,
                                 d, scale, int(bool(causal)), _dtype_code(q), _stream(stream)))
     return o, lse
+
+
+def attn_bwd_varlen(q, k, v, o, lse, dout, cu_seqlens_q, cu_seqlens_k, max_seqlen_q, max_seqlen_k, causal=False,
+                    scale=None, workspace=None, dq=None, dk=None, dv=None, stream=None):
+    """Backward of attn_fwd_varlen: dq like q [Tq,Hq,d], dk/dv like k/v [Tk,Hkv,d]."""
+    Tq, Hq, d = q.shape
+    Tk, Hkv = k.shape[0], k.shape[1]
+    if cu_seqlens_q.dtype != torch.int32 or cu_seqlens_k.dtype != torch.int32:
+        raise AttnError("cu_seqlens must be int32")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if workspace is None:
+        workspace = torch.empty(attn_bwd_workspace_size(1, Hq, Tq, d), device=q.device, dtype=torch.uint8)
+    _check(_lib.attn_bwd_varlen(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(o, "o"), _dev(lse, "lse"),
+                                _dev(dout, "dout"), _dev(dq, "dq"), _dev(dk, "dk"), _dev(dv, "dv"),
+                                _dev(cu_seqlens_q, "cu_seqlens_q"), _dev(cu_seqlens_k, "cu_seqlens_k"),
+                                cu_seqlens_q.numel() - 1, int(max_seqlen_q), int(max_seqlen_k), Tq, Tk, Hq, Hkv, d,
+                                scale, int(bool(causal)), _dev(workspace, "workspace"),
+                                workspace.numel() * workspace.element_size(), _dtype_code(q), _stream(stream)))
+    return dq, dk, dv
 
 
 def attn_naive_scratch_size(n_q, n_k) -> int:

@@ -200,7 +200,10 @@ namespace {
 int bwd_impl(const void* q, const void* k, const void* v, const float* bias, long long bias_batch_stride,
              const float* alibi, const void* o, const float* lse, const void* dout, void* dq, void* dk, void* dv,
              void* workspace, size_t workspace_bytes, int batch, int h_q, int h_kv, int n_q, int n_k, int d,
-             float scale, int causal, int window_left, int window_right, int dtype, void* stream) {
+             float scale, int causal, int window_left, int window_right, int dtype, void* stream,
+             const int* cu_q = nullptr, const int* cu_k = nullptr, int num_seqs = 0, int max_nq = 0,
+             int max_nk = 0) {
+  // packed sequences: batch 1 of n_q / n_k total rows, cu_q / cu_k prefix offsets
   int rc = check_common(batch, h_q, h_kv, n_q, n_k, d, dtype);
   if (rc) return rc;
   if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return ATTN_ERR_INVALID;
@@ -231,6 +234,8 @@ int bwd_impl(const void* q, const void* k, const void* v, const float* bias, lon
     p.bias_bstride = bias_batch_stride;
     p.lse_bstride = (long long)h_q * n_q;
     p.lse_hstride = n_q;
+    p.cu_q = cu_q;
+    p.cu_k = cu_k;
     p.Hq = h_q;
     p.Hkv = h_kv;
     p.Nq = n_q;
@@ -241,7 +246,8 @@ int bwd_impl(const void* q, const void* k, const void* v, const float* bias, lon
     p.window_right = window_right;
     p.scale = scale;
     return launch_bwd_f32(p, static_cast<const float*>(dout), Drow, static_cast<float*>(dq), static_cast<float*>(dk),
-                          static_cast<float*>(dv), batch, n_q, n_k, st);
+                          static_cast<float*>(dv), cu_q ? num_seqs : batch, cu_q ? max_nq : n_q,
+                          cu_q ? max_nk : n_k, st);
   }
   TcGeom g{};
   g.q = q;
@@ -260,6 +266,11 @@ int bwd_impl(const void* q, const void* k, const void* v, const float* bias, lon
   g.bias = bias;
   g.bias_bstride = bias_batch_stride;
   g.alibi = alibi;
+  g.cu_q = cu_q;
+  g.cu_k = cu_k;
+  g.num_seqs = num_seqs;
+  g.max_nq = max_nq;
+  g.max_nk = max_nk;
   return launch_bwd_sm100(g, static_cast<const __nv_bfloat16*>(o), lse, static_cast<const __nv_bfloat16*>(dout),
                           static_cast<__nv_bfloat16*>(dq), static_cast<__nv_bfloat16*>(dk),
                           static_cast<__nv_bfloat16*>(dv), dq_acc, Drow, st);
@@ -292,6 +303,18 @@ int attn_bwd_local(const void* q, const void* k, const void* v, const float* ali
                    int causal, int window_left, int window_right, int dtype, void* stream) {
   return bwd_impl(q, k, v, nullptr, 0, alibi_slopes, o, lse, dout, dq, dk, dv, workspace, workspace_bytes, batch,
                   h_q, h_kv, n_q, n_k, d, scale, causal, window_left, window_right, dtype, stream);
+}
+
+int attn_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+                    void* dq, void* dk, void* dv, const int* cu_seqlens_q, const int* cu_seqlens_k, int num_seqs,
+                    int max_seqlen_q, int max_seqlen_k, int total_q, int total_k, int h_q, int h_kv, int d,
+                    float scale, int causal, void* workspace, size_t workspace_bytes, int dtype, void* stream) {
+  if (num_seqs <= 0 || max_seqlen_q <= 0 || max_seqlen_k <= 0 || !cu_seqlens_q || !cu_seqlens_k)
+    return ATTN_ERR_INVALID;
+  if (max_seqlen_q > total_q || max_seqlen_k > total_k) return ATTN_ERR_INVALID;
+  return bwd_impl(q, k, v, nullptr, 0, nullptr, o, lse, dout, dq, dk, dv, workspace, workspace_bytes, 1, h_q, h_kv,
+                  total_q, total_k, d, scale, causal, -1, -1, dtype, stream, cu_seqlens_q, cu_seqlens_k, num_seqs,
+                  max_seqlen_q, max_seqlen_k);
 }
 
 int attn_splitkv_num_splits(int batch, int h_q, int n_q, int n_k) {

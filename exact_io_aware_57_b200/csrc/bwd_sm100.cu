@@ -8,7 +8,8 @@
 //
 // Three launches:
 //   bwd_pre    D_i = dO_i . O_i (fp32) and zero the fp32 dQ accumulator
-//   bwd_main   one CTA per (128-key tile, KV head, batch); K_j and V_j stay in
+//   bwd_main   one CTA per (128-key tile, KV head, batch or packed sequence);
+//              K_j and V_j stay in
 //              shared memory, dK_j and dV_j accumulate in TMEM over every query
 //              tile and every query head of the group
 //   bwd_dq     dQ = scale * accumulator -> bf16
@@ -78,6 +79,8 @@ struct BwdParams {
   const float* bias;
   long long bias_bstride;
   const float* alibi;
+  const int* cu_q;  // packed sequences: prefix offsets (device), or null
+  const int* cu_k;
   int Hq, Hkv, Nq, Nk;
   float scale, scale_log2;
   int causal;
@@ -238,9 +241,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   Smem& s = *reinterpret_cast<Smem*>(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  const int n_tile = blockIdx.x, hk = blockIdx.y, b = blockIdx.z;
+  const int n_tile = blockIdx.x, hk = blockIdx.y;
   const int n0 = n_tile * BN;
-  const int len_q = p.Nq, len_k = p.Nk;
+  // dense: batch element b; packed: sequence blockIdx.z at rows q_off / k_off of batch 0
+  int b = blockIdx.z, q_off = 0, k_off = 0, len_q = p.Nq, len_k = p.Nk;
+  if (p.cu_q) {
+    q_off = p.cu_q[blockIdx.z];
+    len_q = p.cu_q[blockIdx.z + 1] - q_off;
+    k_off = p.cu_k[blockIdx.z];
+    len_k = p.cu_k[blockIdx.z + 1] - k_off;
+    b = 0;
+  }
+  if (n0 >= len_k) return;  // past this sequence's keys: uniform, before any barrier or TMEM use
   const int diag = len_k - len_q;  // query i is aligned with key i + diag
   const int G = p.Hq / p.Hkv;
   // query rows that see at least one key of n0 .. n0 + BN - 1
@@ -292,7 +304,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int c = 0; c < D / 32; ++c)
           tma_reduce_add_4d(&tm_dq, (c < kBoxes ? s.q[st] : s.dout[st]) + (c % kBoxes) * (128 * 128), c * 32, h,
-                            i0, b);
+                            q_off + i0, b);
         bulk_commit();
         bulk_wait_read0();
       }
@@ -310,8 +322,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_expect_tx(&s.kv_full, 2 * Smem::kTileBytes);
 #pragma unroll
         for (int kb = 0; kb < KB; ++kb) {
-          tma_load_4d(s.k + kb * BN * 128, &tm_k, &s.kv_full, kb * 64, hk, n0, b);
-          tma_load_4d(s.v + kb * BN * 128, &tm_v, &s.kv_full, kb * 64, hk, n0, b);
+          tma_load_4d(s.k + kb * BN * 128, &tm_k, &s.kv_full, kb * 64, hk, k_off + n0, b);
+          tma_load_4d(s.v + kb * BN * 128, &tm_v, &s.kv_full, kb * 64, hk, k_off + n0, b);
         }
       }
     }
@@ -322,7 +334,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int i0 = (i_first + step % per_head) * BM;
       // LSE / D rows of this step into registers first (their latency overlaps
       // the wait for the stage)
-      const long long row0 = ((long long)b * p.Hq + h) * p.Nq;
+      const long long row0 = ((long long)b * p.Hq + h) * p.Nq + q_off;
       float l2v[BM / 32], drv[BM / 32];
 #pragma unroll
       for (int e = 0; e < BM / 32; ++e) {
@@ -340,8 +352,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_expect_tx(&s.q_full[st], 2 * Smem::kTileBytes);
 #pragma unroll
         for (int kb = 0; kb < KB; ++kb) {
-          tma_load_4d(s.q[st] + kb * BM * 128, &tm_q, &s.q_full[st], kb * 64, h, i0, b);
-          tma_load_4d(s.dout[st] + kb * BM * 128, &tm_do, &s.q_full[st], kb * 64, h, i0, b);
+          tma_load_4d(s.q[st] + kb * BM * 128, &tm_q, &s.q_full[st], kb * 64, h, q_off + i0, b);
+          tma_load_4d(s.dout[st] + kb * BM * 128, &tm_do, &s.q_full[st], kb * 64, h, q_off + i0, b);
         }
       }
 #pragma unroll
@@ -490,7 +502,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok && n_steps > 0) ok = __all_sync(0xffffffffu, mbar_wait(&s.drain, 0, ab));
     tc_fence_after();
     if (ok) {
-      const long long row = (((long long)b * p.Nk + kj) * p.Hkv + hk) * D + grp * (D / 2);
+      const long long row = (((long long)b * p.Nk + k_off + kj) * p.Hkv + hk) * D + grp * (D / 2);
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         const uint32_t col0 = (half == 0 ? kColDV : kColDK) + grp * (D / 2);
@@ -575,7 +587,7 @@ int launch_main_t(const TcGeom& g, const CUtensorMap& mq, const CUtensorMap& mk,
   auto kern = bwd_main_kernel<D, BIAS>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return ATTN_ERR_CUDA;
-  dim3 grid((g.Nk + BN - 1) / BN, g.Hkv, g.B);
+  dim3 grid(((g.cu_q ? g.max_nk : g.Nk) + BN - 1) / BN, g.Hkv, g.cu_q ? g.num_seqs : g.B);
   record_kernel_event(ATTN_KERNEL_BWD, 0, st);
   kern<<<grid, kThreads, smem, st>>>(mq, mk, mv, mdo, mdq, p);
   record_kernel_event(ATTN_KERNEL_BWD, 1, st);
@@ -588,7 +600,7 @@ int launch_main_t(const TcGeom& g, const CUtensorMap& mq, const CUtensorMap& mk,
 int launch_bwd_sm100(const TcGeom& g, const __nv_bfloat16* o, const float* lse, const __nv_bfloat16* dout,
                      __nv_bfloat16* dq, __nv_bfloat16* dk, __nv_bfloat16* dv, float* dq_acc, float* Drow,
                      cudaStream_t st) {
-  if (g.cu_q) return ATTN_ERR_UNSUPPORTED;
+  // packed sequences are one batch of g.Nq / g.Nk total rows
   // 1) D and zeroed accumulator
   {
     const long long rows = (long long)g.B * g.Nq * g.Hq;
@@ -629,6 +641,8 @@ int launch_bwd_sm100(const TcGeom& g, const __nv_bfloat16* o, const float* lse, 
   p.bias = g.bias;
   p.bias_bstride = g.bias_bstride;
   p.alibi = g.alibi;
+  p.cu_q = g.cu_q;
+  p.cu_k = g.cu_k;
   p.Hq = g.Hq;
   p.Hkv = g.Hkv;
   p.Nq = g.Nq;

@@ -127,6 +127,19 @@ int attn_bwd_local(const void* q, const void* k, const void* v, const float* ali
                    int dtype, void* stream);
 
 /*
+ * Backward of attn_fwd_varlen (packed sequences, same layouts and offsets):
+ * o, lse and dout as attn_fwd_varlen produced / consumed them; dq like q,
+ * dk / dv like k / v.  workspace: DEVICE, 256-byte aligned,
+ * attn_bwd_workspace_size(1, h_q, total_q, d) bytes.  Causal masking applies
+ * inside each sequence; no bias.  Otherwise as attn_bwd.
+ */
+int attn_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                    const void* dout, void* dq, void* dk, void* dv, const int* cu_seqlens_q,
+                    const int* cu_seqlens_k, int num_seqs, int max_seqlen_q, int max_seqlen_k,
+                    int total_q, int total_k, int h_q, int h_kv, int d, float scale, int causal,
+                    void* workspace, size_t workspace_bytes, int dtype, void* stream);
+
+/*
  * Split-KV forward: the keys are cut into num_splits contiguous ranges (whole
  * 128-key tiles); each (query tile, head, batch, split) is an independent CTA
  * that writes the exact attention of its rows over its own keys (O_t fp32,

@@ -48,6 +48,24 @@ def rel_fro(a, b) -> float:
     return float(np.linalg.norm(a - b) / max(1e-30, np.linalg.norm(b)))
 
 
+def check_grad(name, got, ref, dtype=torch.bfloat16):
+    """One gradient against the oracle: max-abs for fp32, relative Frobenius for
+    bf16.  A gradient that vanishes exactly in the definition (one visible key
+    per row: P = 1, so dS = P (dP - D) = 0 and dQ = dK = 0) has no relative
+    error to speak of; there only rounding noise may remain (max-abs 1e-3)."""
+    got = np.asarray(got, dtype=np.float64)
+    if dtype == torch.float32:
+        e = max_abs(got, ref)
+        assert e <= TOL_F32, f"{name} max-abs {e:.3e} > {TOL_F32}"
+    elif not np.asarray(ref).any():
+        e = max_abs(got, ref)
+        assert e <= 1e-3, f"{name} should vanish, max-abs {e:.3e}"
+    else:
+        e = rel_fro(got, ref)
+        assert e <= TOL_GRAD_BF16, f"{name} rel Frobenius {e:.3e} > {TOL_GRAD_BF16}"
+    return e
+
+
 def gpu_fwd(inp, causal, scale=None, bias=None, alibi=None):
     from exact_io_aware_57_b200 import attn
 
