@@ -296,7 +296,7 @@ def make_job(w, args, dev, rank):
         if w.splitkv:
             t = args.num_splits or attn.attn_splitkv_num_splits(w.batch, w.h_q, n_q, w.n)
             j.splits = t
-            sws = torch.empty(max(256, attn._lib.attn_splitkv_workspace_size(w.batch, w.h_q, n_q, w.d, t)),
+            sws = torch.empty(max(256, attn.attn_splitkv_workspace_size(w.batch, w.h_q, n_q, w.d, t)),
                               device=dev, dtype=torch.uint8)
 
         def step():

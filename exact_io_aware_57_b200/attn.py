@@ -173,6 +173,10 @@ def attn_splitkv_num_splits(batch, h_q, n_q, n_k) -> int:
     return int(_lib.attn_splitkv_num_splits(batch, h_q, n_q, n_k))
 
 
+def attn_splitkv_workspace_size(batch, h_q, n_q, d, num_splits) -> int:
+    return int(_lib.attn_splitkv_workspace_size(batch, h_q, n_q, d, num_splits))
+
+
 def attn_fwd_splitkv(q, k, v, causal=False, scale=None, num_splits=0, out=None, lse=None, workspace=None,
                      stream=None):
     """attn_fwd computed over num_splits key ranges and merged (bf16, dense)."""
@@ -183,7 +187,7 @@ def attn_fwd_splitkv(q, k, v, causal=False, scale=None, num_splits=0, out=None, 
     lse = torch.empty((B, Hq, Nq), device=q.device, dtype=torch.float32) if lse is None else lse
     t = int(num_splits) if num_splits and num_splits > 0 else attn_splitkv_num_splits(B, Hq, Nq, Nk)
     if workspace is None:
-        workspace = torch.empty(max(256, int(_lib.attn_splitkv_workspace_size(B, Hq, Nq, d, t))), device=q.device,
+        workspace = torch.empty(max(256, attn_splitkv_workspace_size(B, Hq, Nq, d, t)), device=q.device,
                                 dtype=torch.uint8)
     _check(_lib.attn_fwd_splitkv(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(o, "o"), _dev(lse, "lse"), B, Hq,
                                  Hkv, Nq, Nk, d, scale, int(bool(causal)), t, _dev(workspace, "workspace"),
