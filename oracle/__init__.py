@@ -77,8 +77,8 @@ class Oracle:
         L = self._lib
         i, d, ll = ctypes.c_int, ctypes.c_double, ctypes.c_longlong
         P = _c_dbl_p
-        L.oracle_attn_fwd.argtypes = [P, P, P, P, ll, P, P, i, i, i, i, i, i, d, i, i, i]
-        L.oracle_attn_fwd_rows.argtypes = [P, P, P, P, ctypes.POINTER(ll), i, P, P, i, i, i, d, i, i, i]
+        L.oracle_attn_fwd.argtypes = [P, P, P, P, ll, P, P, i, i, i, i, i, i, i, d, i, i, i]
+        L.oracle_attn_fwd_rows.argtypes = [P, P, P, P, ctypes.POINTER(ll), i, P, P, i, i, i, i, d, i, i, i]
         L.oracle_attn_fwd_varlen.argtypes = [P, P, P, ctypes.POINTER(ctypes.c_int),
                                              ctypes.POINTER(ctypes.c_int), i, P, P, i, i, i, d, i, i, i]
         L.oracle_attn_fwd_stream.argtypes = [P, P, P, P, ll, P, P, i, i, i, i, i, i, d, i, i, i, i,
@@ -108,13 +108,13 @@ class Oracle:
         unbounded on that side)."""
         q, k, v = _f64(q), _f64(k), _f64(v)
         B, Nq, Hq, d = q.shape
-        Nk, Hkv = k.shape[1], k.shape[2]
+        Nk, Hkv, dv = k.shape[1], k.shape[2], v.shape[3]
         scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
         b, bstride = self._bias(bias, Hq, Nq, Nk)
-        o = np.zeros((B, Nq, Hq, d))
+        o = np.zeros((B, Nq, Hq, dv))
         lse = np.zeros((B, Hq, Nq))
         self._lib.oracle_attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(b) if b is not None else None,
-                                  bstride, _ptr(o), _ptr(lse), B, Hq, Hkv, Nq, Nk, d, scale,
+                                  bstride, _ptr(o), _ptr(lse), B, Hq, Hkv, Nq, Nk, d, dv, scale,
                                   int(bool(causal)), *_window(window))
         return o, lse
 
@@ -138,16 +138,16 @@ class Oracle:
         rows: query indices of q_rows; bias_rows [R,Nk] or None."""
         q_rows, k_head, v_head = _f64(q_rows), _f64(k_head), _f64(v_head)
         R, d = q_rows.shape
-        Nk = k_head.shape[0]
+        Nk, dv = k_head.shape[0], v_head.shape[1]
         scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
         rows = np.ascontiguousarray(np.asarray(rows, dtype=np.int64))
         br = _f64(bias_rows) if bias_rows is not None else None
-        o = np.zeros((R, d))
+        o = np.zeros((R, dv))
         lse = np.zeros(R)
         self._lib.oracle_attn_fwd_rows(_ptr(q_rows), _ptr(k_head), _ptr(v_head),
                                        _ptr(br) if br is not None else None,
                                        rows.ctypes.data_as(ctypes.POINTER(ctypes.c_longlong)), R,
-                                       _ptr(o), _ptr(lse), int(Nq), Nk, d, scale, int(bool(causal)),
+                                       _ptr(o), _ptr(lse), int(Nq), Nk, d, dv, scale, int(bool(causal)),
                                        *_window(window))
         return o, lse
 

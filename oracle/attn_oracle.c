@@ -34,6 +34,9 @@
  *
  * Layouts (row-major, innermost last):
  *   q, o, dout, dq : [B, Nq, Hq, d]      k, v, dk, dv : [B, Nk, Hkv, d]
+ *   (the forward also takes a value width dv != d: v [B, Nk, Hkv, dv] and
+ *   o [B, Nq, Hq, dv], "Understanding FlashAttention Pt 1", 0.2 Notation, which
+ *   gives V its own width d_v)
  *   lse            : [B, Hq, Nq]         bias         : [Hq, Nq, Nk] + b * bias_bstride
  *
  * ORACLE_MUTANT (compile-time, default 0) plants one known mistake; the test
@@ -122,24 +125,24 @@ static double row_scores(const double* qi, const double* kbase, long long kstrid
  * scores, subtract the max, exponentiate, normalise).  p[] receives the
  * normalised probabilities of the visible keys when non-NULL.
  */
-static void fwd_row(const double* qi, const double* kbase, const double* vbase,
-                    long long kvstride, const double* brow, long long nvis, int d,
+static void fwd_row(const double* qi, const double* kbase, long long kstride, const double* vbase,
+                    long long vstride, const double* brow, long long nvis, int d, int dv,
                     double scale, double* s, double* p, double* oi, double* lse_i) {
-  for (int c = 0; c < d; ++c) oi[c] = 0.0;
+  for (int c = 0; c < dv; ++c) oi[c] = 0.0;
   if (nvis == 0) { *lse_i = -INFINITY; return; }
-  double m = row_scores(qi, kbase, kvstride, brow, nvis, d, scale, s);
+  double m = row_scores(qi, kbase, kstride, brow, nvis, d, scale, s);
   if (m == -INFINITY) { *lse_i = -INFINITY; if (p) for (long long j = 0; j < nvis; ++j) p[j] = 0.0; return; }
   double l = 0.0;
   for (long long j = 0; j < nvis; ++j) { s[j] = exp(s[j] - m); l += s[j]; }
   for (long long j = 0; j < nvis; ++j) {
     const double w = s[j] / l;
     if (p) p[j] = w;
-    const double* vj = vbase + j * kvstride;
+    const double* vj = vbase + j * vstride;
 #if ORACLE_MUTANT == 10
-    const double* kj = kbase + j * kvstride; /* planted: K used in place of V */
-    for (int c = 0; c < d; ++c) oi[c] += w * kj[c];
+    const double* kj = kbase + j * kstride; /* planted: K used in place of V */
+    for (int c = 0; c < dv; ++c) oi[c] += w * kj[c % d];
 #else
-    for (int c = 0; c < d; ++c) oi[c] += w * vj[c];
+    for (int c = 0; c < dv; ++c) oi[c] += w * vj[c];
 #endif
   }
 #if ORACLE_MUTANT == 5
@@ -152,7 +155,7 @@ static void fwd_row(const double* qi, const double* kbase, const double* vbase,
 void oracle_attn_fwd(const double* q, const double* k, const double* v,
                      const double* bias, long long bias_bstride,
                      double* o, double* lse, int B, int Hq, int Hkv, int Nq, int Nk,
-                     int d, double scale, int causal, int wl, int wr) {
+                     int d, int dv, double scale, int causal, int wl, int wr) {
   const long long nbh = (long long)B * Hq;
 #pragma omp parallel
   {
@@ -162,14 +165,15 @@ void oracle_attn_fwd(const double* q, const double* k, const double* v,
       const int b = (int)(bh / Hq), h = (int)(bh % Hq);
       const int hk = kv_head_of(h, Hq, Hkv);
       const double* kb = k + idx4(b, 0, hk, 0, Nk, Hkv, d);
-      const double* vb = v + idx4(b, 0, hk, 0, Nk, Hkv, d);
+      const double* vb = v + idx4(b, 0, hk, 0, Nk, Hkv, dv);
       for (long long i = 0; i < Nq; ++i) {
         const double* brow = bias ? bias + b * bias_bstride + ((long long)h * Nq + i) * Nk : NULL;
         long long lo;
         const long long nvis = key_range(i, Nq, Nk, causal, wl, wr, &lo);
-        const long long kvs = (long long)Hkv * d;
-        fwd_row(q + idx4(b, i, h, 0, Nq, Hq, d), kb + lo * kvs, vb + lo * kvs, kvs, brow ? brow + lo : NULL,
-                nvis, d, scale, s, NULL, o + idx4(b, i, h, 0, Nq, Hq, d), lse + ((long long)b * Hq + h) * Nq + i);
+        const long long ks = (long long)Hkv * d, vs = (long long)Hkv * dv;
+        fwd_row(q + idx4(b, i, h, 0, Nq, Hq, d), kb + lo * ks, ks, vb + lo * vs, vs, brow ? brow + lo : NULL,
+                nvis, d, dv, scale, s, NULL, o + idx4(b, i, h, 0, Nq, Hq, dv),
+                lse + ((long long)b * Hq + h) * Nq + i);
       }
     }
     free(s);
@@ -184,7 +188,7 @@ void oracle_attn_fwd(const double* q, const double* k, const double* v,
  */
 void oracle_attn_fwd_rows(const double* q_rows, const double* k_head, const double* v_head,
                           const double* bias_rows, const long long* rows, int R,
-                          double* o_rows, double* lse_rows, int Nq, int Nk, int d,
+                          double* o_rows, double* lse_rows, int Nq, int Nk, int d, int dv,
                           double scale, int causal, int wl, int wr) {
 #pragma omp parallel
   {
@@ -193,9 +197,9 @@ void oracle_attn_fwd_rows(const double* q_rows, const double* k_head, const doub
     for (int r = 0; r < R; ++r) {
       long long lo;
       const long long nvis = key_range(rows[r], Nq, Nk, causal, wl, wr, &lo);
-      fwd_row(q_rows + (long long)r * d, k_head + lo * d, v_head + lo * d, d,
-              bias_rows ? bias_rows + (long long)r * Nk + lo : NULL, nvis, d, scale, s, NULL,
-              o_rows + (long long)r * d, lse_rows + r);
+      fwd_row(q_rows + (long long)r * d, k_head + lo * d, d, v_head + lo * dv, dv,
+              bias_rows ? bias_rows + (long long)r * Nk + lo : NULL, nvis, d, dv, scale, s, NULL,
+              o_rows + (long long)r * dv, lse_rows + r);
     }
     free(s);
   }
@@ -227,7 +231,7 @@ void oracle_attn_fwd_varlen(const double* q, const double* k, const double* v,
         long long lo;
         const long long nvis = key_range(i, nq, nk, causal, wl, wr, &lo);
         const long long kvs = (long long)Hkv * d;
-        fwd_row(q + ((q0 + i) * Hq + h) * d, kb + lo * kvs, vb + lo * kvs, kvs, NULL, nvis, d, scale, s,
+        fwd_row(q + ((q0 + i) * Hq + h) * d, kb + lo * kvs, kvs, vb + lo * kvs, kvs, NULL, nvis, d, d, scale, s,
                 NULL, o + ((q0 + i) * Hq + h) * d, lse + (long long)h * Tq + q0 + i);
       }
     }
@@ -341,7 +345,7 @@ void oracle_attn_bwd(const double* q, const double* k, const double* v,
           const long long nvis = key_range(i, Nq, Nk, causal, wl, wr, &lo);
           const long long kvs = (long long)Hkv * d;
           double lse_i;
-          fwd_row(qi, kb + lo * kvs, vb + lo * kvs, kvs, brow ? brow + lo : NULL, nvis, d, scale, s, p, oi,
+          fwd_row(qi, kb + lo * kvs, kvs, vb + lo * kvs, kvs, brow ? brow + lo : NULL, nvis, d, d, scale, s, p, oi,
                   &lse_i);
           for (int c = 0; c < d; ++c) dqi[c] = 0.0;
           if (lse_i == -INFINITY) continue;

@@ -268,7 +268,33 @@ def pin_window_slices(orc):
     return worst <= 1e-13, f"max abs err {worst:.2e}"
 
 
+def pin_value_width(orc):
+    """V with its own width d_v != d (the handbook's 0.2 Notation gives V a
+    separate width): every row equals scipy's softmax of its scaled scores
+    times V, for d_v = 12 and 3 against d = 8, causal and not, GQA 4:2."""
+    rng = np.random.default_rng(22)
+    worst = 0.0
+    B, nq, nk, hq, hkv, d = 2, 6, 9, 4, 2, 8
+    for dv in (12, 3):
+        for causal in (False, True):
+            q = _rand(rng, B, nq, hq, d)
+            k = _rand(rng, B, nk, hkv, d)
+            v = _rand(rng, B, nk, hkv, dv)
+            o, l = orc.fwd(q, k, v, causal=causal)
+            if o.shape != (B, nq, hq, dv):
+                return False, f"output shape {o.shape}"
+            for b in range(B):
+                for h in range(hq):
+                    for i in range(nq):
+                        last = nk - 1 if not causal else i + (nk - nq)
+                        s_ = q[b, i, h] @ k[b, :last + 1, h // 2].T / math.sqrt(d)
+                        worst = max(worst, float(np.max(np.abs(o[b, i, h] - softmax(s_) @ v[b, :last + 1, h // 2]))),
+                                    abs(float(l[b, h, i] - logsumexp(s_))))
+    return worst <= 1e-13, f"max abs err {worst:.2e}"
+
+
 ALL_PINS = {
+    "value_width": pin_value_width,
     "window_slices": pin_window_slices,
     "merge_every_split": pin_merge_every_split,
     "stream_equals_oneshot": pin_stream_equals_oneshot,
