@@ -40,6 +40,7 @@ EXPORTS = {
                             _F, _I, _I, _I, _I, _VP]),
     "attn_bwd_varlen": (_I, [_VP, _VP, _VP, _VP, _FP, _VP, _VP, _VP, _VP, _IP, _IP, _I, _I, _I, _I, _I, _I, _I, _I,
                              _F, _I, _VP, _SZ, _I, _VP]),
+    "attn_fwd_dv": (_I, [_VP, _VP, _VP, _VP, _FP, _I, _I, _I, _I, _I, _I, _I, _F, _I, _I, _VP]),
     "attn_splitkv_num_splits": (_I, [_I, _I, _I, _I]),
     "attn_splitkv_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
     "attn_fwd_splitkv": (_I, [_VP, _VP, _VP, _VP, _FP, _I, _I, _I, _I, _I, _I, _F, _I, _I, _VP, _SZ, _I, _VP]),
@@ -166,6 +167,18 @@ def attn_fwd(q, k, v, bias=None, causal=False, scale=None, out=None, lse=None, s
     bp, bs = _bias_args(bias, B, Hq, Nq, Nk)
     _check(_lib.attn_fwd(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), bp, bs, _dev(o, "o"), _dev(lse, "lse"),
                          B, Hq, Hkv, Nq, Nk, d, scale, int(bool(causal)), _dtype_code(q), _stream(stream)))
+    return o, lse
+
+
+def attn_fwd_dv(q, k, v, causal=False, scale=None, out=None, lse=None, stream=None):
+    """Forward with V of its own width: q/k [..., d], v [B,Nk,Hkv,d_v] -> o [B,Nq,Hq,d_v]."""
+    B, Nq, Hq, d = q.shape
+    Nk, Hkv, dv = k.shape[1], k.shape[2], v.shape[3]
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    o = torch.empty((B, Nq, Hq, dv), device=q.device, dtype=q.dtype) if out is None else out
+    lse = torch.empty((B, Hq, Nq), device=q.device, dtype=torch.float32) if lse is None else lse
+    _check(_lib.attn_fwd_dv(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(o, "o"), _dev(lse, "lse"), B, Hq, Hkv,
+                            Nq, Nk, d, dv, scale, int(bool(causal)), _dtype_code(q), _stream(stream)))
     return o, lse
 
 

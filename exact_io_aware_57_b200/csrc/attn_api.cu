@@ -317,6 +317,34 @@ int attn_bwd_varlen(const void* q, const void* k, const void* v, const void* o, 
                   max_seqlen_q, max_seqlen_k);
 }
 
+int attn_fwd_dv(const void* q, const void* k, const void* v, void* o, float* lse, int batch, int h_q, int h_kv,
+                int n_q, int n_k, int d, int d_v, float scale, int causal, int dtype, void* stream) {
+  int rc = check_common(batch, h_q, h_kv, n_q, n_k, d, dtype);
+  if (rc) return rc;
+  if (d_v != 64 && d_v != 128) return ATTN_ERR_UNSUPPORTED;
+  if (d_v == d)
+    return fwd_impl(q, k, v, nullptr, 0, nullptr, o, lse, batch, h_q, h_kv, n_q, n_k, d, scale, causal, -1, -1,
+                    dtype, stream);
+  if (dtype != ATTN_BF16) return ATTN_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return ATTN_ERR_INVALID;
+  if (!supported_device()) return ATTN_ERR_UNSUPPORTED;
+  TcGeom g{};
+  g.q = q;
+  g.k = k;
+  g.v = v;
+  g.B = batch;
+  g.Hq = h_q;
+  g.Hkv = h_kv;
+  g.Nq = n_q;
+  g.Nk = n_k;
+  g.D = d;
+  g.Dv = d_v;
+  g.causal = causal != 0;
+  g.scale = scale;
+  return launch_fwd_sm100(g, static_cast<__nv_bfloat16*>(o), lse, static_cast<cudaStream_t>(stream));
+}
+
 int attn_splitkv_num_splits(int batch, int h_q, int n_q, int n_k) {
   if (batch <= 0 || h_q <= 0 || n_q <= 0 || n_k <= 0) return 1;
   const long long ctas = (long long)((n_q + 127) / 128) * h_q * batch;

@@ -44,21 +44,23 @@ namespace {
 
 constexpr int BM = 128;          // query rows per CTA
 constexpr int BN = 128;          // keys per KV tile
-// K/V shared-memory stages: as many as fit beside the Q tile in 227 KB
-template <int D>
-constexpr int kStages = D == 64 ? 4 : 3;
+// K/V shared-memory stages: as many as fit beside the Q tile in 227 KB (at
+// most four).  DV is the width of V and O (d_v), D that of Q and K.
+template <int D, int DV>
+constexpr int kStages = (D == 128 && DV == 128) ? 3 : 4;
 constexpr int kThreads = 192;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColS = 0, kColO = 256, kColP = 384;
 constexpr float kRescaleThreshold = 8.f;  // log2 units: P stays <= 256
 
-template <int D>
+template <int D, int DV>
 struct FwdSmem {
-  static constexpr int NST = kStages<D>;
-  static constexpr int kTileBytes = BM * D * 2;  // 128 rows x D bf16
+  static constexpr int NST = kStages<D, DV>;
+  static constexpr int kTileBytes = BM * D * 2;    // 128 rows x D bf16 (Q, K)
+  static constexpr int kVTileBytes = BN * DV * 2;  // 128 rows x DV bf16 (V)
   alignas(1024) uint8_t q[kTileBytes];
   alignas(1024) uint8_t k[NST][kTileBytes];
-  alignas(1024) uint8_t v[NST][kTileBytes];
+  alignas(1024) uint8_t v[NST][kVTileBytes];
   uint64_t q_full;
   uint64_t k_full[NST], k_empty[NST], v_full[NST], v_empty[NST];
   uint64_t s_full[2], p_full[2];
@@ -95,11 +97,11 @@ ATTN_DEVINL void reg_fence(uint32_t (&r)[N]) {
   for (int i = 0; i < N; ++i) asm volatile("" : "+r"(r[i]));
 }
 
-template <int D, int BIAS, bool FAST, bool PARTIAL>
+template <int D, int DV, int BIAS, bool FAST, bool PARTIAL>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_sm100_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
-  using Smem = FwdSmem<D>;
+  using Smem = FwdSmem<D, DV>;
   constexpr int NST = Smem::NST;
   constexpr int KB = D / 64;  // 64-column (128-byte) blocks per row
   extern __shared__ uint8_t smem_raw[];
@@ -178,9 +180,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           tma_load_4d(s.k[st] + kb * BN * 128, &tm_k, &s.k_full[st], kb * 64, hk, k_off + (j_first + j) * BN, bidx);
         ++issued_k;
         if (!mbar_wait(&s.v_empty[st], ph ^ 1, ab)) break;
-        mbar_expect_tx(&s.v_full[st], Smem::kTileBytes);
+        mbar_expect_tx(&s.v_full[st], Smem::kVTileBytes);
 #pragma unroll
-        for (int kb = 0; kb < KB; ++kb)
+        for (int kb = 0; kb < DV / 64; ++kb)
           tma_load_4d(s.v[st] + kb * BN * 128, &tm_v, &s.v_full[st], kb * 64, hk, k_off + (j_first + j) * BN, bidx);
         ++issued_v;
       }
@@ -197,7 +199,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ===================================================== MMA issuer
     if (lane == 0 && n_kv > 0) {
       constexpr uint32_t idesc_s = idesc_bf16(BM, BN, 0, 0);   // Q: K-major, K_j: K-major
-      constexpr uint32_t idesc_pv = idesc_bf16(BM, D, 0, 1);   // P: TMEM, V_j: MN-major
+      constexpr uint32_t idesc_pv = idesc_bf16(BM, DV, 0, 1);  // P: TMEM, V_j: MN-major
       const uint32_t q_addr = smem_u32(s.q);
       auto issue_s = [&](int j) -> bool {
         const int buf = j & 1, st = j % NST;
@@ -337,7 +339,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         if (__any_sync(0xffffffffu, alpha != 1.f)) {
 #pragma unroll 1
-          for (int c = 0; c < D / 32; ++c) {
+          for (int c = 0; c < DV / 32; ++c) {
             uint32_t orr[32];
             tmem_ld32(tmem + lane_off + kColO + c * 32, orr);
             tmem_wait_ld();
@@ -360,12 +362,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     if (ok) {
       const float inv_l = l > 0.f ? 1.f / l : 0.f;
-      __nv_bfloat16* orow = p.o + bidx * p.o_bstride + ((long long)(q_off + i) * p.Hq + h) * D;
+      __nv_bfloat16* orow = p.o + bidx * p.o_bstride + ((long long)(q_off + i) * p.Hq + h) * DV;
       float* prow = nullptr;
       if constexpr (PARTIAL) prow = p.o_part + split * p.part_o_stride + bidx * p.o_bstride +
-                                    ((long long)(q_off + i) * p.Hq + h) * D;
+                                    ((long long)(q_off + i) * p.Hq + h) * DV;
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) {
+      for (int c = 0; c < DV / 32; ++c) {
         uint32_t orr[32];
         if (n_kv > 0) {
           tmem_ld32(tmem + lane_off + kColO + c * 32, orr);
@@ -416,13 +418,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D, int BIAS, bool FAST, bool PARTIAL = false>
+template <int D, int DV, int BIAS, bool FAST, bool PARTIAL = false>
 int launch_fwd_t(const TcGeom& g, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                  const FwdParams& p, cudaStream_t st) {
   // At least half of the SM's shared memory, so that a second CTA never waits
   // on the 512 TMEM columns this one holds.
-  const size_t smem = std::max<size_t>(sizeof(FwdSmem<D>) + 1024, 116 * 1024);
-  auto kern = fwd_sm100_kernel<D, BIAS, FAST, PARTIAL>;
+  const size_t smem = std::max<size_t>(sizeof(FwdSmem<D, DV>) + 1024, 116 * 1024);
+  auto kern = fwd_sm100_kernel<D, DV, BIAS, FAST, PARTIAL>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return ATTN_ERR_CUDA;
   const int max_nq = g.cu_q ? g.max_nq : g.Nq;
@@ -439,6 +441,7 @@ int launch_fwd_t(const TcGeom& g, const CUtensorMap& mq, const CUtensorMap& mk, 
 int launch_fwd_sm100(const TcGeom& g, __nv_bfloat16* o, float* lse, cudaStream_t st, const SplitKV* split) {
   // 4-D views (d, head, row, batch); packed inputs are one batch of `total` rows.
   const int B = g.cu_q ? 1 : g.B;
+  const int dv = g.Dv ? g.Dv : g.D;  // width of V and O
   CUtensorMap mq, mk, mv;
   const uint32_t box[4] = {64, 1, 128, 1};
   {
@@ -450,7 +453,9 @@ int launch_fwd_sm100(const TcGeom& g, __nv_bfloat16* o, float* lse, cudaStream_t
     const uint64_t dims[4] = {(uint64_t)g.D, (uint64_t)g.Hkv, (uint64_t)g.Nk, (uint64_t)B};
     const uint64_t str[3] = {(uint64_t)g.D * 2, (uint64_t)g.Hkv * g.D * 2, (uint64_t)g.Nk * g.Hkv * g.D * 2};
     if (encode_tmap_bf16(&mk, g.k, 4, dims, str, box) != ATTN_OK) return ATTN_ERR_CUDA;
-    if (encode_tmap_bf16(&mv, g.v, 4, dims, str, box) != ATTN_OK) return ATTN_ERR_CUDA;
+    const uint64_t dv_dims[4] = {(uint64_t)dv, (uint64_t)g.Hkv, (uint64_t)g.Nk, (uint64_t)B};
+    const uint64_t dv_str[3] = {(uint64_t)dv * 2, (uint64_t)g.Hkv * dv * 2, (uint64_t)g.Nk * g.Hkv * dv * 2};
+    if (encode_tmap_bf16(&mv, g.v, 4, dv_dims, dv_str, box) != ATTN_OK) return ATTN_ERR_CUDA;
   }
   FwdParams p{};
   p.o = o;
@@ -464,7 +469,7 @@ int launch_fwd_sm100(const TcGeom& g, __nv_bfloat16* o, float* lse, cudaStream_t
   p.Hkv = g.Hkv;
   p.Nq = g.Nq;
   p.Nk = g.Nk;
-  p.o_bstride = g.cu_q ? 0 : (long long)g.Nq * g.Hq * g.D;
+  p.o_bstride = g.cu_q ? 0 : (long long)g.Nq * g.Hq * dv;
   p.lse_bstride = g.cu_q ? 0 : (long long)g.Hq * g.Nq;
   p.lse_hstride = g.Nq;  // packed: Nq is the total row count
   p.scale_log2 = g.scale * kLog2e;
@@ -486,23 +491,31 @@ int launch_fwd_sm100(const TcGeom& g, __nv_bfloat16* o, float* lse, cudaStream_t
   if (!p.status) return ATTN_ERR_CUDA;
   // FAST: no bias and a positive scale, so the row max can be taken on raw scores
   const bool fast = !g.bias && !g.alibi && g.scale > 0.f;
+  if (dv != g.D) {  // value width of its own: dense or packed, no bias, one pass
+    if (split || g.bias || g.alibi) return ATTN_ERR_UNSUPPORTED;
+    if (g.D == 128)
+      return fast ? launch_fwd_t<128, 64, kBiasNone, true>(g, mq, mk, mv, p, st)
+                  : launch_fwd_t<128, 64, kBiasNone, false>(g, mq, mk, mv, p, st);
+    return fast ? launch_fwd_t<64, 128, kBiasNone, true>(g, mq, mk, mv, p, st)
+                : launch_fwd_t<64, 128, kBiasNone, false>(g, mq, mk, mv, p, st);
+  }
   if (split) {  // no bias on this path
     if (g.D == 64)
-      return fast ? launch_fwd_t<64, kBiasNone, true, true>(g, mq, mk, mv, p, st)
-                  : launch_fwd_t<64, kBiasNone, false, true>(g, mq, mk, mv, p, st);
-    return fast ? launch_fwd_t<128, kBiasNone, true, true>(g, mq, mk, mv, p, st)
-                : launch_fwd_t<128, kBiasNone, false, true>(g, mq, mk, mv, p, st);
+      return fast ? launch_fwd_t<64, 64, kBiasNone, true, true>(g, mq, mk, mv, p, st)
+                  : launch_fwd_t<64, 64, kBiasNone, false, true>(g, mq, mk, mv, p, st);
+    return fast ? launch_fwd_t<128, 128, kBiasNone, true, true>(g, mq, mk, mv, p, st)
+                : launch_fwd_t<128, 128, kBiasNone, false, true>(g, mq, mk, mv, p, st);
   }
   if (g.D == 64) {
-    if (g.bias) return launch_fwd_t<64, kBiasDense, false>(g, mq, mk, mv, p, st);
-    if (g.alibi) return launch_fwd_t<64, kBiasAlibi, false>(g, mq, mk, mv, p, st);
-    return fast ? launch_fwd_t<64, kBiasNone, true>(g, mq, mk, mv, p, st)
-                : launch_fwd_t<64, kBiasNone, false>(g, mq, mk, mv, p, st);
+    if (g.bias) return launch_fwd_t<64, 64, kBiasDense, false>(g, mq, mk, mv, p, st);
+    if (g.alibi) return launch_fwd_t<64, 64, kBiasAlibi, false>(g, mq, mk, mv, p, st);
+    return fast ? launch_fwd_t<64, 64, kBiasNone, true>(g, mq, mk, mv, p, st)
+                : launch_fwd_t<64, 64, kBiasNone, false>(g, mq, mk, mv, p, st);
   }
-  if (g.bias) return launch_fwd_t<128, kBiasDense, false>(g, mq, mk, mv, p, st);
-  if (g.alibi) return launch_fwd_t<128, kBiasAlibi, false>(g, mq, mk, mv, p, st);
-  return fast ? launch_fwd_t<128, kBiasNone, true>(g, mq, mk, mv, p, st)
-              : launch_fwd_t<128, kBiasNone, false>(g, mq, mk, mv, p, st);
+  if (g.bias) return launch_fwd_t<128, 128, kBiasDense, false>(g, mq, mk, mv, p, st);
+  if (g.alibi) return launch_fwd_t<128, 128, kBiasAlibi, false>(g, mq, mk, mv, p, st);
+  return fast ? launch_fwd_t<128, 128, kBiasNone, true>(g, mq, mk, mv, p, st)
+              : launch_fwd_t<128, 128, kBiasNone, false>(g, mq, mk, mv, p, st);
 }
 
 }  // namespace attn

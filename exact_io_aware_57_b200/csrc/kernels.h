@@ -69,6 +69,7 @@ struct TcGeom {
   long long bias_bstride;
   const float* alibi;          // per-query-head ALiBi slopes (device) or null
   int window_left = -1, window_right = -1;  // local attention sizes; negative: unbounded
+  int Dv = 0;                  // width of V and O when it differs from D (forward only), else 0
 };
 
 // Split-KV forward: keys cut into num_splits ranges of split_len (a multiple of

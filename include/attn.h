@@ -127,6 +127,18 @@ int attn_bwd_local(const void* q, const void* k, const void* v, const float* ali
                    int dtype, void* stream);
 
 /*
+ * Forward with a value width of its own ("Understanding FlashAttention Pt 1",
+ * 0.2 Notation: V and O have d_v columns, Q and K have d): v is
+ * [batch, n_k, h_kv, d_v] and o is [batch, n_q, h_q, d_v], d and d_v each in
+ * {64, 128}.  d_v == d is attn_fwd without a bias; d_v != d takes bf16 only
+ * (ATTN_ERR_UNSUPPORTED for fp32) and has no backward in this library.
+ * Otherwise as attn_fwd.
+ */
+int attn_fwd_dv(const void* q, const void* k, const void* v, void* o, float* lse, int batch,
+                int h_q, int h_kv, int n_q, int n_k, int d, int d_v, float scale, int causal,
+                int dtype, void* stream);
+
+/*
  * Backward of attn_fwd_varlen (packed sequences, same layouts and offsets):
  * o, lse and dout as attn_fwd_varlen produced / consumed them; dq like q,
  * dk / dv like k / v.  workspace: DEVICE, 256-byte aligned,
