@@ -104,6 +104,8 @@ int check_common(int batch, int h_q, int h_kv, int n_q, int n_k, int d, int dtyp
   // the kernels index rows with 32-bit coordinates (TMA) and 64-bit offsets
   if ((long long)batch * n_q > (1ll << 31) - 1 || (long long)batch * n_k > (1ll << 31) - 1) return ATTN_ERR_INVALID;
   if (n_q > kMaxSeqLen || n_k > kMaxSeqLen) return ATTN_ERR_UNSUPPORTED;
+  // grid y runs over heads and z over batch elements (times key splits): 65535 at most
+  if (h_q > 65535 || batch > 65535) return ATTN_ERR_UNSUPPORTED;
   return ATTN_OK;
 }
 
@@ -377,11 +379,12 @@ int attn_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float
   if (dtype != ATTN_BF16) return ATTN_ERR_UNSUPPORTED;
   if (!q || !k || !v || !o || !lse) return ATTN_ERR_INVALID;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return ATTN_ERR_INVALID;
-  if (!supported_device()) return ATTN_ERR_UNSUPPORTED;
   if (num_splits <= 0) num_splits = attn_splitkv_num_splits(batch, h_q, n_q, n_k);
   const int kv_tiles = (n_k + 127) / 128;
   const int tiles_per_split = (kv_tiles + std::min(num_splits, kv_tiles) - 1) / std::min(num_splits, kv_tiles);
   const int splits = (kv_tiles + tiles_per_split - 1) / tiles_per_split;  // none of them empty
+  if ((long long)batch * splits > 65535) return ATTN_ERR_UNSUPPORTED;     // grid z
+  if (!supported_device()) return ATTN_ERR_UNSUPPORTED;
   TcGeom g{};
   g.q = q;
   g.k = k;

@@ -53,7 +53,8 @@ extern "C" {
 
 #define ATTN_OK 0
 #define ATTN_ERR_INVALID (-1)     /* null pointer, bad size, h_q % h_kv != 0, misaligned */
-#define ATTN_ERR_UNSUPPORTED (-2) /* d not in {64,128}, a sequence over 2^28 rows, no sm_100 device */
+#define ATTN_ERR_UNSUPPORTED (-2) /* d not in {64,128}, a sequence over 2^28 rows, over 65535 heads or
+                                     batch elements, no sm_100 device */
 #define ATTN_ERR_WORKSPACE (-3)   /* workspace missing or smaller than attn_bwd_workspace_size */
 #define ATTN_ERR_CUDA (-4)        /* a CUDA runtime/driver call failed */
 #define ATTN_ERR_TIMEOUT (-5)     /* a kernel gave up a bounded wait (device status word) */

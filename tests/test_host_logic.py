@@ -46,7 +46,8 @@ def test_split_workspace_size():
 
 
 @pytest.mark.parametrize("entry", ["fwd_local", "bwd_local", "fwd_alibi_null", "splitkv_f32", "merge_dim",
-                                   "merge_null", "bwd_varlen_null", "bwd_varlen_maxlen"])
+                                   "merge_null", "bwd_varlen_null", "bwd_varlen_maxlen", "grid_heads",
+                                   "grid_batch_splits"])
 def test_new_entry_points_validate_before_launch(entry):
     attn, lib = _lib()
     p = ctypes.c_void_p(256)  # never dereferenced: validation fails first
@@ -76,10 +77,16 @@ def test_new_entry_points_validate_before_launch(entry):
         rc = lib.attn_bwd_varlen(p, p, p, p, fp, p, p, p, p, None, ip, 2, 64, 64, 128, 128, 4, 4, 128, 0.1, 1, p,
                                  1 << 20, 0, None)
         want = attn.ATTN_ERR_INVALID
-    else:                         # longest sequence longer than the packed total
+    elif entry == "bwd_varlen_maxlen":  # longest sequence longer than the packed total
         rc = lib.attn_bwd_varlen(p, p, p, p, fp, p, p, p, p, ip, ip, 2, 200, 64, 128, 128, 4, 4, 128, 0.1, 1, p,
                                  1 << 20, 0, None)
         want = attn.ATTN_ERR_INVALID
+    elif entry == "grid_heads":   # more heads than the grid's y extent
+        rc = lib.attn_fwd(p, p, p, None, 0, p, fp, 1, 70000, 70000, 64, 64, 128, 0.1, 0, 0, None)
+        want = attn.ATTN_ERR_UNSUPPORTED
+    else:                         # batch x key splits beyond the grid's z extent
+        rc = lib.attn_fwd_splitkv(p, p, p, p, fp, 20000, 1, 1, 64, 4096, 128, 0.1, 0, 8, p, 1 << 40, 0, None)
+        want = attn.ATTN_ERR_UNSUPPORTED
     assert rc == want
     assert attn.attn_launch_count() == before
 
