@@ -41,6 +41,7 @@ EXPORTS = {
     "attn_bwd_varlen": (_I, [_VP, _VP, _VP, _VP, _FP, _VP, _VP, _VP, _VP, _IP, _IP, _I, _I, _I, _I, _I, _I, _I, _I,
                              _F, _I, _VP, _SZ, _I, _VP]),
     "attn_fwd_dv": (_I, [_VP, _VP, _VP, _VP, _FP, _I, _I, _I, _I, _I, _I, _I, _F, _I, _I, _VP]),
+    "attn_selftest_wait_timeout": (_I, [ctypes.c_longlong, _VP]),
     "attn_splitkv_num_splits": (_I, [_I, _I, _I, _I]),
     "attn_splitkv_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
     "attn_fwd_splitkv": (_I, [_VP, _VP, _VP, _VP, _FP, _I, _I, _I, _I, _I, _I, _F, _I, _I, _VP, _SZ, _I, _VP]),
@@ -180,6 +181,11 @@ def attn_fwd_dv(q, k, v, causal=False, scale=None, out=None, lse=None, stream=No
     _check(_lib.attn_fwd_dv(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(o, "o"), _dev(lse, "lse"), B, Hq, Hkv,
                             Nq, Nk, d, dv, scale, int(bool(causal)), _dtype_code(q), _stream(stream)))
     return o, lse
+
+
+def attn_selftest_wait_timeout(limit_cycles=1_000_000, stream=None) -> None:
+    """Launch the bounded-wait self-test (a wait that gives up after limit_cycles)."""
+    _check(_lib.attn_selftest_wait_timeout(int(limit_cycles), _stream(stream)))
 
 
 def attn_splitkv_num_splits(batch, h_q, n_q, n_k) -> int:

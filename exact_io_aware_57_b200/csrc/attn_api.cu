@@ -532,6 +532,12 @@ int attn_device_status(void* stream) {
   return value;
 }
 
+int attn_selftest_wait_timeout(long long limit_cycles, void* stream) {
+  if (limit_cycles < 1000 || limit_cycles > kWaitLimitCycles) return ATTN_ERR_INVALID;
+  if (!supported_device()) return ATTN_ERR_UNSUPPORTED;
+  return launch_wait_selftest(limit_cycles, static_cast<cudaStream_t>(stream));
+}
+
 int attn_set_kernel_events(int which, void* start, void* stop) {
   if (which != ATTN_KERNEL_FWD && which != ATTN_KERNEL_BWD) return ATTN_ERR_INVALID;
   if ((start == nullptr) != (stop == nullptr)) return ATTN_ERR_INVALID;

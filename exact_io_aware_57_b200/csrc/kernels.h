@@ -90,6 +90,10 @@ int launch_bwd_sm100(const TcGeom& g, const __nv_bfloat16* o, const float* lse, 
 int launch_fwd_naive(const TcGeom& g, __nv_bfloat16* o, float* lse, float* s_scratch, __nv_bfloat16* p_scratch,
                      cudaStream_t st);
 
+// One warp that waits on a barrier nothing arrives on, giving up after
+// limit_cycles (the shared bounded-wait failure path).
+int launch_wait_selftest(long long limit_cycles, cudaStream_t st);
+
 // Tensor-map encoding (driver entry point resolved at run time).
 int encode_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,
                      const uint64_t* strides_bytes, const uint32_t* box);

@@ -245,6 +245,15 @@ const char* attn_strerror(int code);
 int attn_device_status(void* stream);
 
 /*
+ * Self-test of the failure path: launches one warp that waits on a barrier
+ * nothing arrives on and gives up after limit_cycles SM cycles (1000 ..
+ * 2e9), exactly as every kernel's bounded waits do; the next
+ * attn_device_status then returns ATTN_ERR_TIMEOUT and the context stays
+ * usable.  No fault, no hang.
+ */
+int attn_selftest_wait_timeout(long long limit_cycles, void* stream);
+
+/*
  * Kernel launches issued by this library on the calling host thread since the
  * last reset (reset = 1 clears after reading).  Lets callers count the GPU
  * work of a timed region.

@@ -47,7 +47,7 @@ def test_split_workspace_size():
 
 @pytest.mark.parametrize("entry", ["fwd_local", "bwd_local", "fwd_alibi_null", "splitkv_f32", "merge_dim",
                                    "merge_null", "bwd_varlen_null", "bwd_varlen_maxlen", "grid_heads",
-                                   "grid_batch_splits"])
+                                   "grid_batch_splits", "selftest_limit"])
 def test_new_entry_points_validate_before_launch(entry):
     attn, lib = _lib()
     p = ctypes.c_void_p(256)  # never dereferenced: validation fails first
@@ -84,6 +84,9 @@ def test_new_entry_points_validate_before_launch(entry):
     elif entry == "grid_heads":   # more heads than the grid's y extent
         rc = lib.attn_fwd(p, p, p, None, 0, p, fp, 1, 70000, 70000, 64, 64, 128, 0.1, 0, 0, None)
         want = attn.ATTN_ERR_UNSUPPORTED
+    elif entry == "selftest_limit":  # wait limit below the accepted range
+        rc = lib.attn_selftest_wait_timeout(10, None)
+        want = attn.ATTN_ERR_INVALID
     else:                         # batch x key splits beyond the grid's z extent
         rc = lib.attn_fwd_splitkv(p, p, p, p, fp, 20000, 1, 1, 64, 4096, 128, 0.1, 0, 8, p, 1 << 40, 0, None)
         want = attn.ATTN_ERR_UNSUPPORTED
