@@ -30,8 +30,15 @@ def _rand(rng, *shape, scale=1.0):
 
 
 def _rel(a, b):
-    a, b = np.asarray(a), np.asarray(b)
-    return float(np.max(np.abs(a - b)) / max(1e-300, np.max(np.abs(b))))
+    """Max relative error; a mismatch in non-finite entries (e.g. -inf against a
+    finite value) counts as an infinite error."""
+    a, b = np.asarray(a, dtype=np.float64), np.asarray(b, dtype=np.float64)
+    fa, fb = np.isfinite(a), np.isfinite(b)
+    if not np.array_equal(fa, fb) or not np.array_equal(a[~fa], b[~fb]):
+        return float("inf")
+    if not fa.any():
+        return 0.0
+    return float(np.max(np.abs(a[fa] - b[fb])) / max(1e-300, np.max(np.abs(b[fb]))))
 
 
 def pin_merge_every_split(orc):
