@@ -313,6 +313,7 @@ int attn_bwd_varlen(const void* q, const void* k, const void* v, const void* o, 
                     float scale, int causal, void* workspace, size_t workspace_bytes, int dtype, void* stream) {
   if (num_seqs <= 0 || max_seqlen_q <= 0 || max_seqlen_k <= 0 || !cu_seqlens_q || !cu_seqlens_k)
     return ATTN_ERR_INVALID;
+  if (num_seqs > 65535) return ATTN_ERR_UNSUPPORTED;  // grid z runs over sequences
   if (max_seqlen_q > total_q || max_seqlen_k > total_k) return ATTN_ERR_INVALID;
   return bwd_impl(q, k, v, nullptr, 0, nullptr, o, lse, dout, dq, dk, dv, workspace, workspace_bytes, 1, h_q, h_kv,
                   total_q, total_k, d, scale, causal, -1, -1, dtype, stream, cu_seqlens_q, cu_seqlens_k, num_seqs,
@@ -429,6 +430,7 @@ int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float*
                     const int* cu_seqlens_k, int num_seqs, int max_seqlen_q, int max_seqlen_k, int total_q,
                     int total_k, int h_q, int h_kv, int d, float scale, int causal, int dtype, void* stream) {
   if (num_seqs <= 0 || max_seqlen_q <= 0 || max_seqlen_k <= 0) return ATTN_ERR_INVALID;
+  if (num_seqs > 65535) return ATTN_ERR_UNSUPPORTED;  // grid z runs over sequences
   int rc = check_common(1, h_q, h_kv, total_q, total_k, d, dtype);
   if (rc) return rc;
   if (!q || !k || !v || !o || !lse || !cu_seqlens_q || !cu_seqlens_k) return ATTN_ERR_INVALID;

@@ -47,7 +47,7 @@ def test_split_workspace_size():
 
 @pytest.mark.parametrize("entry", ["fwd_local", "bwd_local", "fwd_alibi_null", "splitkv_f32", "merge_dim",
                                    "merge_null", "bwd_varlen_null", "bwd_varlen_maxlen", "grid_heads",
-                                   "grid_batch_splits", "selftest_limit"])
+                                   "grid_batch_splits", "selftest_limit", "grid_seqs"])
 def test_new_entry_points_validate_before_launch(entry):
     attn, lib = _lib()
     p = ctypes.c_void_p(256)  # never dereferenced: validation fails first
@@ -83,6 +83,10 @@ def test_new_entry_points_validate_before_launch(entry):
         want = attn.ATTN_ERR_INVALID
     elif entry == "grid_heads":   # more heads than the grid's y extent
         rc = lib.attn_fwd(p, p, p, None, 0, p, fp, 1, 70000, 70000, 64, 64, 128, 0.1, 0, 0, None)
+        want = attn.ATTN_ERR_UNSUPPORTED
+    elif entry == "grid_seqs":    # more packed sequences than the grid's z extent
+        rc = lib.attn_fwd_varlen(p, p, p, p, fp, ip, ip, 70000, 64, 64, 1 << 20, 1 << 20, 4, 4, 128, 0.1, 1, 0,
+                                 None)
         want = attn.ATTN_ERR_UNSUPPORTED
     elif entry == "selftest_limit":  # wait limit below the accepted range
         rc = lib.attn_selftest_wait_timeout(10, None)
