@@ -85,6 +85,8 @@ class Oracle:
                                              ctypes.POINTER(ll)]
         L.oracle_attn_bwd.argtypes = [P, P, P, P, ll, P, P, P, P, i, i, i, i, i, i, d, i, i, i]
         L.oracle_merge_partials.argtypes = [P, P, i, i, i, P, P]
+        L.oracle_quantize_e4m3.argtypes = [P, ll, d, P]
+        L.oracle_quantize_e4m3.restype = None
         for f in (L.oracle_attn_fwd, L.oracle_attn_fwd_rows, L.oracle_attn_fwd_varlen,
                   L.oracle_attn_fwd_stream, L.oracle_attn_bwd, L.oracle_merge_partials):
             f.restype = None
@@ -182,6 +184,14 @@ class Oracle:
                                   bstride, _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
                                   B, Hq, Hkv, Nq, Nk, d, scale, int(bool(causal)), *_window(window))
         return dq, dk, dv
+
+    # --------------------------------------------------------------------- fp8
+    def quantize_e4m3(self, x, scale=1.0):
+        """Dequantised e4m3 values of x / scale, times scale (fp64, same shape)."""
+        x = _f64(x)
+        out = np.empty_like(x)
+        self._lib.oracle_quantize_e4m3(_ptr(x), x.size, float(scale), _ptr(out))
+        return out
 
     # -------------------------------------------------------------------- merge
     def merge_partials(self, o_parts, lse_parts):

@@ -385,6 +385,33 @@ void oracle_attn_bwd(const double* q, const double* k, const double* v,
 }
 
 /*
+ * FP8 inputs (the handbook's contents name FlashAttention-3's FP8 path, 5.4 to
+ * 5.6, without a definition): the oracle for an FP8 forward is the exact
+ * attention of the quantised-then-dequantised inputs, so only the rounding to
+ * e4m3 is defined here.  e4m3 (the OCP 8-bit floating-point format): 4
+ * exponent bits with bias 7, 3 mantissa bits, no infinities, largest finite
+ * value 448, subnormals m * 2^-9.  Rounding is to nearest with ties to an even
+ * mantissa; magnitudes at or above 448 saturate to 448.  out = q(x / scale) *
+ * scale for a positive per-tensor scale.
+ */
+static double round_e4m3(double x) {
+  if (x != x) return x;
+  const double a = fabs(x);
+  if (a >= 448.0) return copysign(448.0, x);
+  int ex;
+  frexp(a, &ex);                              /* a = f * 2^ex, f in [0.5, 1) */
+  int e = ex - 1;                             /* a in [2^e, 2^(e+1)) */
+  if (a == 0.0 || e < -6) e = -6;             /* subnormal range: same spacing as 2^-6 */
+  const double spacing = ldexp(1.0, e - 3);   /* 3 mantissa bits */
+  const double r = nearbyint(a / spacing);    /* default rounding mode: ties to even */
+  return copysign(r * spacing, x);
+}
+
+void oracle_quantize_e4m3(const double* x, long long n, double scale, double* out) {
+  for (long long i = 0; i < n; ++i) out[i] = round_e4m3(x[i] / scale) * scale;
+}
+
+/*
  * Merge of partial results over disjoint key shards: shard t holds the exact
  * attention (o_t, lse_t) of the row over its own keys only.  The combined row
  * follows from the same rescale-and-add recurrence as the streaming forward:
