@@ -216,6 +216,9 @@ int attn_bwd_noalloc(const void* q, const void* k, const void* v, const float* b
  * arrays of num_seqs + 1 non-decreasing prefix offsets starting at 0; sequence z
  * owns rows cu[z] .. cu[z+1]-1.  max_seqlen_q / max_seqlen_k bound the lengths
  * (they size the launch).  Causal masking applies inside each sequence.  No bias.
+ * The offsets live in device memory and are not read on the host: offsets that
+ * decrease, exceed the totals or a length above max_seqlen are the caller's
+ * error, and the results are then undefined.
  */
 int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
                     const int* cu_seqlens_q, const int* cu_seqlens_k, int num_seqs,
