@@ -83,7 +83,7 @@ class Oracle:
                                              ctypes.POINTER(ctypes.c_int), i, P, P, i, i, i, d, i, i, i]
         L.oracle_attn_fwd_stream.argtypes = [P, P, P, P, ll, P, P, i, i, i, i, i, i, d, i, i, i, i,
                                              ctypes.POINTER(ll)]
-        L.oracle_attn_bwd.argtypes = [P, P, P, P, ll, P, P, P, P, i, i, i, i, i, i, d, i, i, i]
+        L.oracle_attn_bwd.argtypes = [P, P, P, P, ll, P, P, P, P, i, i, i, i, i, i, i, d, i, i, i]
         L.oracle_merge_partials.argtypes = [P, P, i, i, i, P, P]
         L.oracle_quantize_e4m3.argtypes = [P, ll, d, P]
         L.oracle_quantize_e4m3.restype = None
@@ -174,7 +174,7 @@ class Oracle:
         """dQ, dK, dV of the forward above for upstream gradient dout (fp64)."""
         q, k, v, dout = _f64(q), _f64(k), _f64(v), _f64(dout)
         B, Nq, Hq, d = q.shape
-        Nk, Hkv = k.shape[1], k.shape[2]
+        Nk, Hkv, dvw = k.shape[1], k.shape[2], v.shape[3]
         scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
         b, bstride = self._bias(bias, Hq, Nq, Nk)
         dq = np.zeros_like(q)
@@ -182,7 +182,7 @@ class Oracle:
         dv = np.zeros_like(v)
         self._lib.oracle_attn_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(b) if b is not None else None,
                                   bstride, _ptr(dout), _ptr(dq), _ptr(dk), _ptr(dv),
-                                  B, Hq, Hkv, Nq, Nk, d, scale, int(bool(causal)), *_window(window))
+                                  B, Hq, Hkv, Nq, Nk, d, dvw, scale, int(bool(causal)), *_window(window))
         return dq, dk, dv
 
     # --------------------------------------------------------------------- fp8

@@ -316,16 +316,17 @@ void oracle_attn_fwd_stream(const double* q, const double* k, const double* v,
 void oracle_attn_bwd(const double* q, const double* k, const double* v,
                      const double* bias, long long bias_bstride, const double* dout,
                      double* dq, double* dk, double* dv, int B, int Hq, int Hkv, int Nq,
-                     int Nk, int d, double scale, int causal, int wl, int wr) {
+                     int Nk, int d, int dvw, double scale, int causal, int wl, int wr) {
+  /* dvw: width of V, O, dO and dV (d_v); d: width of Q, K, dQ and dK */
   const int G = Hq / Hkv;
   const long long nbk = (long long)B * Hkv;
   memset(dk, 0, sizeof(double) * (size_t)B * Nk * Hkv * d);
-  memset(dv, 0, sizeof(double) * (size_t)B * Nk * Hkv * d);
+  memset(dv, 0, sizeof(double) * (size_t)B * Nk * Hkv * dvw);
 #pragma omp parallel
   {
     double* s = (double*)malloc(sizeof(double) * (Nk > 0 ? Nk : 1));
     double* p = (double*)malloc(sizeof(double) * (Nk > 0 ? Nk : 1));
-    double* oi = (double*)malloc(sizeof(double) * d);
+    double* oi = (double*)malloc(sizeof(double) * dvw);
 #pragma omp for schedule(dynamic, 1)
     for (long long bk = 0; bk < nbk; ++bk) {
       const int b = (int)(bk / Hkv), hk = (int)(bk % Hkv);
@@ -335,38 +336,38 @@ void oracle_attn_bwd(const double* q, const double* k, const double* v,
         h = g * Hkv + hk; /* planted: interleaved groups (matches kv_head_of above) */
 #endif
         const double* kb = k + idx4(b, 0, hk, 0, Nk, Hkv, d);
-        const double* vb = v + idx4(b, 0, hk, 0, Nk, Hkv, d);
+        const double* vb = v + idx4(b, 0, hk, 0, Nk, Hkv, dvw);
         for (long long i = 0; i < Nq; ++i) {
           const double* qi = q + idx4(b, i, h, 0, Nq, Hq, d);
-          const double* doi = dout + idx4(b, i, h, 0, Nq, Hq, d);
+          const double* doi = dout + idx4(b, i, h, 0, Nq, Hq, dvw);
           double* dqi = dq + idx4(b, i, h, 0, Nq, Hq, d);
           const double* brow = bias ? bias + b * bias_bstride + ((long long)h * Nq + i) * Nk : NULL;
           long long lo;
           const long long nvis = key_range(i, Nq, Nk, causal, wl, wr, &lo);
-          const long long kvs = (long long)Hkv * d;
+          const long long kvs = (long long)Hkv * d, vvs = (long long)Hkv * dvw;
           double lse_i;
-          fwd_row(qi, kb + lo * kvs, kvs, vb + lo * kvs, kvs, brow ? brow + lo : NULL, nvis, d, d, scale, s, p, oi,
-                  &lse_i);
+          fwd_row(qi, kb + lo * kvs, kvs, vb + lo * vvs, vvs, brow ? brow + lo : NULL, nvis, d, dvw, scale, s, p,
+                  oi, &lse_i);
           for (int c = 0; c < d; ++c) dqi[c] = 0.0;
           if (lse_i == -INFINITY) continue;
           double Di = 0.0;
-          for (int c = 0; c < d; ++c) Di += doi[c] * oi[c];
+          for (int c = 0; c < dvw; ++c) Di += doi[c] * oi[c];
           for (long long j = 0; j < nvis; ++j) { /* key lo + j; p[j] is its probability */
             const double* kj = kb + (lo + j) * kvs;
-            const double* vj = vb + (lo + j) * kvs;
+            const double* vj = vb + (lo + j) * vvs;
             double* dkj = dk + idx4(b, lo + j, hk, 0, Nk, Hkv, d);
-            double* dvj = dv + idx4(b, lo + j, hk, 0, Nk, Hkv, d);
+            double* dvj = dv + idx4(b, lo + j, hk, 0, Nk, Hkv, dvw);
             double dP = 0.0;
-            for (int c = 0; c < d; ++c) dP += doi[c] * vj[c];
+            for (int c = 0; c < dvw; ++c) dP += doi[c] * vj[c];
 #if ORACLE_MUTANT == 6
             const double dS = p[j] * (dP + Di); /* planted: wrong sign */
 #else
             const double dS = p[j] * (dP - Di);
 #endif
 #if ORACLE_MUTANT == 8
-            for (int c = 0; c < d; ++c) dvj[c] += dS * doi[c]; /* planted: dS in place of P */
+            for (int c = 0; c < dvw; ++c) dvj[c] += dS * doi[c]; /* planted: dS in place of P */
 #else
-            for (int c = 0; c < d; ++c) dvj[c] += p[j] * doi[c];
+            for (int c = 0; c < dvw; ++c) dvj[c] += p[j] * doi[c];
 #endif
 #if ORACLE_MUTANT == 7
             for (int c = 0; c < d; ++c) dqi[c] += dS * kj[c]; /* planted: scale dropped */

@@ -192,18 +192,22 @@ def _loss(orc, q, k, v, dout, bias, causal, window=None):
 
 
 def pin_backward_fd(orc):
-    """Central finite differences (step 1e-6) of sum(dO * O) w.r.t. Q, K, V."""
+    """Central finite differences (step 1e-6) of sum(dO * O) w.r.t. Q, K, V,
+    including a value width d_v != d and local windows."""
     rng = np.random.default_rng(19)
     worst = 0.0
-    for (B, nq, nk, hq, hkv, d, causal, use_bias, window) in ((1, 5, 5, 2, 1, 4, True, True, None),
-                                                               (1, 3, 6, 2, 2, 3, False, False, None),
-                                                               (2, 4, 4, 1, 1, 2, True, False, None),
-                                                               (1, 6, 6, 2, 1, 3, True, True, (2, -1)),
-                                                               (1, 5, 7, 1, 1, 2, False, False, (1, 1))):
+    # (B, Nq, Nk, Hq, Hkv, d, d_v, causal, bias, window)
+    for (B, nq, nk, hq, hkv, d, dv_, causal, use_bias, window) in (
+            (1, 5, 5, 2, 1, 4, 4, True, True, None),
+            (1, 3, 6, 2, 2, 3, 3, False, False, None),
+            (2, 4, 4, 1, 1, 2, 2, True, False, None),
+            (1, 6, 6, 2, 1, 3, 3, True, True, (2, -1)),
+            (1, 5, 7, 1, 1, 2, 2, False, False, (1, 1)),
+            (1, 4, 5, 2, 1, 3, 5, True, False, None)):      # value width d_v != d
         q = _rand(rng, B, nq, hq, d)
         k = _rand(rng, B, nk, hkv, d)
-        v = _rand(rng, B, nk, hkv, d)
-        dout = _rand(rng, B, nq, hq, d)
+        v = _rand(rng, B, nk, hkv, dv_)
+        dout = _rand(rng, B, nq, hq, dv_)
         bias = _rand(rng, hq, nq, nk) if use_bias else None
         dq, dk, dv = orc.bwd(q, k, v, dout, bias=bias, causal=causal, window=window)
         for x, g in ((q, dq), (k, dk), (v, dv)):
