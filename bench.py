@@ -542,8 +542,24 @@ def run_reference(args):
     print(json.dumps(line), flush=True)
 
 
+def check_args(args):
+    """Reject options that do not apply to the chosen workload (before any GPU work)."""
+    from exact_io_aware_57_b200 import workloads
+
+    w = workloads.WORKLOADS[args.workload]
+    if args.window is not None and (w.varlen or not w.causal or w.n_q):
+        raise SystemExit("--window applies to the causal dense workloads (c3, c4, c5b)")
+    if args.bias_mode == "alibi" and not w.bias:
+        raise SystemExit("--bias-mode alibi applies to the grouped-query workload c4")
+    if args.with_backward and not w.varlen:
+        raise SystemExit("--with-backward applies to the packed workload c5a")
+    if args.num_splits and not w.splitkv:
+        raise SystemExit("--num-splits applies to the split-KV workload kv1")
+
+
 def main(argv=None):
     args = parse_args(argv)
+    check_args(args)
     if args.impl == "reference":
         run_reference(args)
     else:

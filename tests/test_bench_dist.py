@@ -59,3 +59,16 @@ def test_traffic_record_tracks_kernel_source(tmp_path, monkeypatch):
     assert bench.recorded_traffic() == 12345
     f.write_text("kernel_source_sha256_16: 0000\ndram_bytes_per_full_launch: 12345\n")
     assert bench.recorded_traffic() is None
+
+
+@pytest.mark.parametrize("argv", [["--workload", "c2", "--window", "10"], ["--bias-mode", "alibi"],
+                                  ["--with-backward"], ["--num-splits", "4"]])
+def test_options_outside_their_workload_are_rejected(argv):
+    with pytest.raises(SystemExit):
+        bench.check_args(bench.parse_args(argv))
+
+
+def test_options_on_their_workload_are_accepted():
+    for argv in (["--window", "1024"], ["--workload", "c4", "--bias-mode", "alibi"],
+                 ["--workload", "c5a", "--with-backward"], ["--workload", "kv1", "--num-splits", "8"]):
+        bench.check_args(bench.parse_args(argv))
