@@ -69,18 +69,19 @@ def pin_merge_every_split(orc):
 
 
 def pin_stream_equals_oneshot(orc):
-    """Streaming (m, l, a) replay with every block size equals the one-shot row."""
+    """Streaming (m, l, a) replay with every block size equals the one-shot row
+    (also under local windows, where a row's first block starts mid-sequence)."""
     rng = np.random.default_rng(12)
     worst = 0.0
     q = _rand(rng, 2, 16, 2, 8, scale=2.0)
     k = _rand(rng, 2, 16, 1, 8, scale=2.0)
     v = _rand(rng, 2, 16, 1, 8)
     bias = _rand(rng, 2, 16, 16)
-    for causal in (False, True):
+    for causal, window in ((False, None), (True, None), (True, (5, None)), (False, (3, 2))):
         for b in (None, bias):
-            o_ref, l_ref = orc.fwd(q, k, v, bias=b, causal=causal)
+            o_ref, l_ref = orc.fwd(q, k, v, bias=b, causal=causal, window=window)
             for blk in range(1, 17):
-                o_s, l_s, _ = orc.fwd_stream(q, k, v, bias=b, causal=causal, block=blk)
+                o_s, l_s, _ = orc.fwd_stream(q, k, v, bias=b, causal=causal, block=blk, window=window)
                 worst = max(worst, _rel(o_s, o_ref), _rel(l_s, l_ref))
     return worst <= 1e-13, f"max rel err {worst:.2e}"
 

@@ -66,11 +66,11 @@ def test_varlen_matches_dense(orc):
     q = rng.standard_normal((T, hq, d))
     k = rng.standard_normal((T, hkv, d))
     v = rng.standard_normal((T, hkv, d))
-    for causal in (False, True):
-        o, lse = orc.fwd_varlen(q, k, v, cu, cu, causal=causal)
+    for causal, window in ((False, None), (True, None), (True, (3, None)), (False, (2, 1))):
+        o, lse = orc.fwd_varlen(q, k, v, cu, cu, causal=causal, window=window)
         for z in range(len(lens)):
             a, b = cu[z], cu[z + 1]
-            o_d, l_d = orc.fwd(q[None, a:b], k[None, a:b], v[None, a:b], causal=causal)
+            o_d, l_d = orc.fwd(q[None, a:b], k[None, a:b], v[None, a:b], causal=causal, window=window)
             np.testing.assert_allclose(o[a:b], o_d[0], rtol=0, atol=1e-14)
             np.testing.assert_allclose(lse[:, a:b], l_d[0], rtol=0, atol=1e-13)
 
