@@ -9,9 +9,8 @@
 // Three launches:
 //   bwd_pre    D_i = dO_i . O_i (fp32) and zero the fp32 dQ accumulator
 //   bwd_main   one CTA per (128-key tile, KV head, batch or packed sequence);
-//              K_j and V_j stay in
-//              shared memory, dK_j and dV_j accumulate in TMEM over every query
-//              tile and every query head of the group
+//              K_j and V_j stay in shared memory, dK_j and dV_j accumulate in
+//              TMEM over every query tile and every query head of the group
 //   bwd_dq     dQ = scale * accumulator -> bf16
 //
 // bwd_main roles (10 warps):

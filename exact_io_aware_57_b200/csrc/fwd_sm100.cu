@@ -6,7 +6,7 @@
 // updates the per-row softmax state and the rescaled value sum, then is
 // dropped rather than stored).
 //
-//   warp 0      TMA producer: Q once, then K_j / V_j into a 2-stage smem ring
+//   warp 0      TMA producer: Q once, then K_j / V_j into a 3- or 4-stage smem ring
 //   warp 1      TMEM owner + single-thread tcgen05.mma issuer
 //   warps 2..5  softmax warpgroup: thread t owns query row t (TMEM lane t)
 //
@@ -16,10 +16,12 @@
 //   [384,448) P buffer 0   [448,512) P buffer 1     (bf16 pairs, A operand of P V_j)
 //
 // Per key tile j the softmax thread of row i forms t = s * scale * log2(e)
-// (+ bias * log2(e)), the new running max m' = max(m, max_j t), p = 2^(t - m'),
-// l' = 2^(m - m') l + sum p ("Softmax does not need the matrix", "Carry the
-// Normalizer", in base 2), writes P to TMEM and -- once the previous P V has
-// landed -- rescales the O accumulator by 2^(m - m') when the max moved.  The
+// (+ bias * log2(e)), a reference max m' (moved to max_j t only when that
+// exceeds m by more than 2^8), p = 2^(t - m'), l' = 2^(m - m') l + sum p
+// ("Softmax does not need the matrix", "Carry the Normalizer", in base 2),
+// writes P to TMEM and -- once the previous P V has landed -- rescales the O
+// accumulator by 2^(m - m') when the reference moved.  V and O may have their
+// own width DV (d_v).  The
 // MMA warp then accumulates O += P V_j.  O / l and LSE = (m + log2 l) ln 2 are
 // written once, after the last tile (the division by l happens a single time,
 // as in the same page's lab).

@@ -72,3 +72,12 @@ def test_options_on_their_workload_are_accepted():
     for argv in (["--window", "1024"], ["--workload", "c4", "--bias-mode", "alibi"],
                  ["--workload", "c5a", "--with-backward"], ["--workload", "kv1", "--num-splits", "8"]):
         bench.check_args(bench.parse_args(argv))
+
+
+def test_source_digest_ignores_comments_but_not_code(tmp_path):
+    a, b, c = tmp_path / "a.cu", tmp_path / "b.cu", tmp_path / "c.cu"
+    a.write_text("int f(int x) { return x + 1; }\n")
+    b.write_text("// a note\nint f(int x) {  /* the increment */\n  return x + 1;  // plus one\n}\n")
+    c.write_text("int f(int x) { return x + 2; }\n")
+    assert bench.source_digest(a) == bench.source_digest(b)
+    assert bench.source_digest(a) != bench.source_digest(c)
