@@ -46,6 +46,7 @@ EXPORTS = {
     "attn_splitkv_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
     "attn_fwd_splitkv": (_I, [_VP, _VP, _VP, _VP, _FP, _I, _I, _I, _I, _I, _I, _F, _I, _I, _VP, _SZ, _I, _VP]),
     "attn_merge_partials": (_I, [_FP, _FP, _I, _VP, _FP, _I, _I, _I, _I, _I, _VP]),
+    "attn_fwd_partial": (_I, [_VP, _VP, _VP, _FP, _FP, _I, _I, _I, _I, _I, _I, _F, _I, _I, _VP]),
     "attn_bwd_workspace_size": (_SZ, [_I, _I, _I, _I]),
     "attn_bwd": (_I, [_VP, _VP, _VP, _FP, _LL, _VP, _FP, _VP, _VP, _VP, _VP, _VP, _SZ, _I, _I, _I, _I, _I,
                       _I, _F, _I, _I, _VP]),
@@ -214,6 +215,24 @@ def attn_fwd_splitkv(q, k, v, causal=False, scale=None, num_splits=0, out=None, 
     return o, lse
 
 
+def attn_fwd_partial(q, k, v, causal=False, scale=None, o_part=None, lse_part=None, stream=None):
+    """Unmerged attention of q [B,Nq,Hq,d] over one key block k/v [B,Nk,Hkv,d] (bf16):
+    o_part fp32 [B,Nq,Hq,d] (normalised over the block) and lse_part fp32 [B,Hq,Nq].
+    Causal aligns the block bottom-right.  Partials of disjoint blocks combine
+    with attn_merge_partials."""
+    B, Nq, Hq, d = q.shape
+    Nk, Hkv = k.shape[1], k.shape[2]
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    o_part = torch.empty((B, Nq, Hq, d), device=q.device, dtype=torch.float32) if o_part is None else o_part
+    lse_part = torch.empty((B, Hq, Nq), device=q.device, dtype=torch.float32) if lse_part is None else lse_part
+    if o_part.dtype != torch.float32 or lse_part.dtype != torch.float32:
+        raise AttnError("partials are fp32")
+    _check(_lib.attn_fwd_partial(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(o_part, "o_part"),
+                                 _dev(lse_part, "lse_part"), B, Hq, Hkv, Nq, Nk, d, scale, int(bool(causal)),
+                                 _dtype_code(q), _stream(stream)))
+    return o_part, lse_part
+
+
 def attn_merge_partials(o_parts, lse_parts, out=None, lse=None, out_dtype=torch.bfloat16, stream=None):
     """Merge fp32 partials o_parts [T,B,Nq,Hq,d], lse_parts [T,B,Hq,Nq] over disjoint key ranges."""
     if o_parts.dtype != torch.float32 or lse_parts.dtype != torch.float32:
@@ -330,7 +349,8 @@ def attn_fwd_naive(q, k, v, causal=False, scale=None, scratch=None, stream=None)
 
 
 def attn_device_status(stream=None) -> int:
-    """Synchronise and return/clear the device status word (0 or ATTN_ERR_TIMEOUT)."""
+    """Synchronise and return/clear the device status word: 0, ATTN_ERR_TIMEOUT
+    (a bounded wait gave up) or ATTN_ERR_INVALID (packed offsets rejected)."""
     return int(_lib.attn_device_status(_stream(stream)))
 
 

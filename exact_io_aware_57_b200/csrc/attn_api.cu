@@ -238,6 +238,8 @@ int bwd_impl(const void* q, const void* k, const void* v, const float* bias, lon
     p.lse_hstride = n_q;
     p.cu_q = cu_q;
     p.cu_k = cu_k;
+    p.max_nq = max_nq;
+    p.max_nk = max_nk;
     p.Hq = h_q;
     p.Hkv = h_kv;
     p.Nq = n_q;
@@ -350,7 +352,7 @@ int attn_fwd_dv(const void* q, const void* k, const void* v, void* o, float* lse
 
 int attn_splitkv_num_splits(int batch, int h_q, int n_q, int n_k) {
   if (batch <= 0 || h_q <= 0 || n_q <= 0 || n_k <= 0) return 1;
-  const long long ctas = (long long)((n_q + 127) / 128) * h_q * batch;
+  const long long ctas = (long long)((n_q + 255) / 256) * h_q * batch;  // 256 query rows per CTA
   const int kv_tiles = (n_k + 127) / 128;
   // One CTA per SM at a time (the forward holds all of TMEM): pick the split
   // count whose last wave is fullest, preferring fewer splits (each adds a
@@ -414,6 +416,35 @@ int attn_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float
   return launch_merge(sp.o_part, sp.lse_part, splits, o, lse, batch, h_q, n_q, d, 0, st);
 }
 
+int attn_fwd_partial(const void* q, const void* k, const void* v, float* o_part, float* lse_part, int batch,
+                     int h_q, int h_kv, int n_q, int n_k, int d, float scale, int causal, int dtype, void* stream) {
+  int rc = check_common(batch, h_q, h_kv, n_q, n_k, d, dtype);
+  if (rc) return rc;
+  if (dtype != ATTN_BF16) return ATTN_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !o_part || !lse_part) return ATTN_ERR_INVALID;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o_part)) return ATTN_ERR_INVALID;
+  if (!supported_device()) return ATTN_ERR_UNSUPPORTED;
+  TcGeom g{};
+  g.q = q;
+  g.k = k;
+  g.v = v;
+  g.B = batch;
+  g.Hq = h_q;
+  g.Hkv = h_kv;
+  g.Nq = n_q;
+  g.Nk = n_k;
+  g.D = d;
+  g.causal = causal != 0;
+  g.scale = scale;
+  // one "split" holding every key of the block: the kernel's partial epilogue
+  SplitKV sp;
+  sp.num_splits = 1;
+  sp.split_len = (n_k + 127) / 128 * 128;
+  sp.o_part = o_part;
+  sp.lse_part = lse_part;
+  return launch_fwd_sm100(g, nullptr, nullptr, static_cast<cudaStream_t>(stream), &sp);
+}
+
 int attn_merge_partials(const float* o_parts, const float* lse_parts, int num_parts, void* o, float* lse, int batch,
                         int h_q, int n_q, int d, int out_dtype, void* stream) {
   if (!o_parts || !lse_parts || !o || !lse || num_parts <= 0 || batch <= 0 || h_q <= 0 || n_q <= 0)
@@ -447,6 +478,8 @@ int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float*
     p.lse = lse;
     p.cu_q = cu_seqlens_q;
     p.cu_k = cu_seqlens_k;
+    p.max_nq = max_seqlen_q;
+    p.max_nk = max_seqlen_k;
     p.lse_hstride = total_q;
     p.Hq = h_q;
     p.Hkv = h_kv;

@@ -17,8 +17,9 @@
 //     the kernels zero what must start at zero on every call, so the contents a
 //     previous call left behind do not matter;
 //   * the first call on a device looks up the array's device address
-//     (cudaGetSymbolAddress) with that device current; make that first call
-//     before any stream capture.
+//     (cudaGetSymbolAddress) with that device current and keeps it; make that
+//     first call before any stream capture.  A cudaDeviceReset after it is not
+//     supported (the array may then sit at another address).
 #include <mutex>
 
 #include "common.cuh"

@@ -80,6 +80,7 @@ struct BwdParams {
   const float* alibi;
   const int* cu_q;  // packed sequences: prefix offsets (device), or null
   const int* cu_k;
+  int max_nq, max_nk;  // packed: bounds on the sequence lengths
   int Hq, Hkv, Nq, Nk;
   float scale, scale_log2;
   int causal;
@@ -245,10 +246,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   // dense: batch element b; packed: sequence blockIdx.z at rows q_off / k_off of batch 0
   int b = blockIdx.z, q_off = 0, k_off = 0, len_q = p.Nq, len_k = p.Nk;
   if (p.cu_q) {
-    q_off = p.cu_q[blockIdx.z];
-    len_q = p.cu_q[blockIdx.z + 1] - q_off;
-    k_off = p.cu_k[blockIdx.z];
-    len_k = p.cu_k[blockIdx.z + 1] - k_off;
+    // invalid offsets: reported in the status word, nothing read or written
+    if (!packed_seq(p.cu_q, blockIdx.z, p.Nq, p.max_nq, p.status, q_off, len_q) ||
+        !packed_seq(p.cu_k, blockIdx.z, p.Nk, p.max_nk, p.status, k_off, len_k))
+      return;
     b = 0;
   }
   if (n0 >= len_k) return;  // past this sequence's keys: uniform, before any barrier or TMEM use
@@ -642,6 +643,8 @@ int launch_bwd_sm100(const TcGeom& g, const __nv_bfloat16* o, const float* lse, 
   p.alibi = g.alibi;
   p.cu_q = g.cu_q;
   p.cu_k = g.cu_k;
+  p.max_nq = g.max_nq;
+  p.max_nk = g.max_nk;
   p.Hq = g.Hq;
   p.Hkv = g.Hkv;
   p.Nq = g.Nq;

@@ -85,6 +85,21 @@ ATTN_DEVINL bool mbar_wait_drain(uint64_t* bar, uint32_t parity, long long limit
   return true;
 }
 
+// Offsets of packed sequence z: sequence z owns rows cu[z] .. cu[z+1]-1 of a
+// buffer of `total` rows.  Accepts 0 <= cu[z] <= cu[z+1] <= total with a length
+// of at most max_len; otherwise raises ATTN_ERR_INVALID in the device status
+// word and returns false, and the caller leaves before touching any row.
+ATTN_DEVINL bool packed_seq(const int* cu, int z, int total, int max_len, int* status, int& off, int& len) {
+  const int a = cu[z], b = cu[z + 1];
+  if (a < 0 || b < a || b > total || b - a > max_len) {
+    atomicExch(status, ATTN_ERR_INVALID);
+    return false;
+  }
+  off = a;
+  len = b - a;
+  return true;
+}
+
 // ------------------------------------------------------------------------- TMA
 ATTN_DEVINL void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
@@ -226,6 +241,24 @@ ATTN_DEVINL float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x on the FMA pipe, for x <= 0 (inputs below -126 give about 2^-126).
+// Cody and Waite's range reduction: x = n + f with n = round(x) (added to
+// 1.5 * 2^23, whose low mantissa bits then hold n) and f in [-1/2, 1/2]; 2^f
+// from the degree-3 polynomial of least maximum relative error on [-1/2, 1/2],
+// fitted by the Remez exchange algorithm (ex2_poly_fit.py: relative error
+// 7.5e-5, far below the 2^-9 of the bf16 P it feeds); n goes into the
+// exponent field by an integer add.  Lets a share of the exponentials bypass
+// the MUFU unit.
+ATTN_DEVINL float ex2_poly(float x) {
+  x = fmaxf(x, -126.f);
+  const float t = __fadd_rn(x, 12582912.f);
+  const float f = __fsub_rn(x, __fsub_rn(t, 12582912.f));
+  float p = fmaf(0.0551716685295105f, f, 0.2426111251115799f);
+  p = fmaf(p, f, 0.6932609677314758f);
+  p = fmaf(p, f, 0.9999280571937561f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
 ATTN_DEVINL uint32_t pack_bf16(float lo, float hi) {

@@ -71,26 +71,7 @@ struct FwdSmem {
   int abort_flag;
 };
 
-struct FwdParams {
-  __nv_bfloat16* o;
-  float* lse;
-  const float* bias;
-  long long bias_bstride;
-  const float* alibi;  // per-query-head slopes (BIAS == kBiasAlibi)
-  const int* cu_q;
-  const int* cu_k;
-  int Hq, Hkv, Nq, Nk;
-  long long o_bstride, lse_bstride, lse_hstride;
-  float scale_log2;
-  int causal;
-  int win_l, win_r;  // key j visible from row i iff i + diag - win_l <= j <= i + diag + win_r
-  int num_splits, split_len;           // split-KV (1, unused: one split)
-  float* o_part;                       // [num_splits, B, Nq, Hq, D] fp32, or null: O in bf16 to o
-  float* lse_part;                     // [num_splits, B, Hq, Nq]
-  long long part_o_stride, part_lse_stride;
-  int* status;
-  long long wait_limit;
-};
+
 
 // Keep the compiler from using TMEM-loaded registers before tcgen05.wait::ld.
 template <int N>
@@ -118,10 +99,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int split = PARTIAL ? (int)blockIdx.z % p.num_splits : 0;
   int q_off = 0, len_q = p.Nq, k_off = 0, len_k = p.Nk, bidx = z;
   if (p.cu_q) {
-    q_off = p.cu_q[z];
-    len_q = p.cu_q[z + 1] - q_off;
-    k_off = p.cu_k[z];
-    len_k = p.cu_k[z + 1] - k_off;
+    // invalid offsets: reported in the status word, nothing read or written
+    if (!packed_seq(p.cu_q, z, p.Nq, p.max_nq, p.status, q_off, len_q) ||
+        !packed_seq(p.cu_k, z, p.Nk, p.max_nk, p.status, k_off, len_k))
+      return;
     bidx = 0;
   }
   const int m0 = m_tile * BM;
@@ -467,6 +448,8 @@ int launch_fwd_sm100(const TcGeom& g, __nv_bfloat16* o, float* lse, cudaStream_t
   p.alibi = g.alibi;
   p.cu_q = g.cu_q;
   p.cu_k = g.cu_k;
+  p.max_nq = g.max_nq;
+  p.max_nk = g.max_nk;
   p.Hq = g.Hq;
   p.Hkv = g.Hkv;
   p.Nq = g.Nq;
@@ -493,6 +476,11 @@ int launch_fwd_sm100(const TcGeom& g, __nv_bfloat16* o, float* lse, cudaStream_t
   if (!p.status) return ATTN_ERR_CUDA;
   // FAST: no bias and a positive scale, so the row max can be taken on raw scores
   const bool fast = !g.bias && !g.alibi && g.scale > 0.f;
+#ifndef ATTN_FWD_SINGLE_TILE
+  if (dv != g.D && (split || g.bias || g.alibi)) return ATTN_ERR_UNSUPPORTED;
+  return launch_fwd_pp(g, mq, mk, mv, p, g.bias ? kBiasDense : g.alibi ? kBiasAlibi : kBiasNone, fast,
+                       split != nullptr, st);
+#else
   if (dv != g.D) {  // value width of its own: dense or packed, no bias, one pass
     if (split || g.bias || g.alibi) return ATTN_ERR_UNSUPPORTED;
     if (g.D == 128)
@@ -518,6 +506,7 @@ int launch_fwd_sm100(const TcGeom& g, __nv_bfloat16* o, float* lse, cudaStream_t
   if (g.alibi) return launch_fwd_t<128, 128, kBiasAlibi, false>(g, mq, mk, mv, p, st);
   return fast ? launch_fwd_t<128, 128, kBiasNone, true>(g, mq, mk, mv, p, st)
               : launch_fwd_t<128, 128, kBiasNone, false>(g, mq, mk, mv, p, st);
+#endif
 }
 
 }  // namespace attn

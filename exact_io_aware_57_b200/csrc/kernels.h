@@ -46,6 +46,8 @@ struct F32Params {
   int window_left = -1, window_right = -1;  // local attention sizes; negative: unbounded
   int win_l = kWinNone, win_r = kWinNone;  // folded from causal and the sizes by the launchers
   float scale;
+  int max_nq = 0, max_nk = 0;  // packed: bounds on the sequence lengths (set by the launchers)
+  int* status = nullptr;       // device status word (set by the launchers)
 };
 
 int launch_fwd_f32(const F32Params& p, int num_z, int max_nq, cudaStream_t st);
@@ -79,6 +81,36 @@ struct SplitKV {
   float* o_part;    // [num_splits, B, Nq, Hq, D]
   float* lse_part;  // [num_splits, B, Hq, Nq]
 };
+// Parameters of the tensor-core forward kernels (built by launch_fwd_sm100).
+struct FwdParams {
+  __nv_bfloat16* o;
+  float* lse;
+  const float* bias;
+  long long bias_bstride;
+  const float* alibi;  // per-query-head slopes (BIAS == kBiasAlibi)
+  const int* cu_q;
+  const int* cu_k;
+  int max_nq, max_nk;  // packed: bounds on the sequence lengths
+  int Hq, Hkv, Nq, Nk;
+  long long o_bstride, lse_bstride, lse_hstride;
+  float scale_log2;
+  int causal;
+  int win_l, win_r;  // key j visible from row i iff i + diag - win_l <= j <= i + diag + win_r
+  int num_splits, split_len;           // split-KV (1, unused: one split)
+  float* o_part;                       // [num_splits, B, Nq, Hq, D] fp32, or null: O in bf16 to o
+  float* lse_part;                     // [num_splits, B, Hq, Nq]
+  long long part_o_stride, part_lse_stride;
+  int* status;
+  long long wait_limit;
+};
+
+// Forward with two 128-row query tiles per CTA whose softmax warpgroups
+// alternate on the tensor pipe (fwd_pp_sm100.cu).  fast: no bias and a
+// positive scale (the row max may be taken on raw scores); partial: split-KV
+// partials to p.o_part / p.lse_part.
+int launch_fwd_pp(const TcGeom& g, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                  const FwdParams& p, int bias_kind, bool fast, bool partial, cudaStream_t st);
+
 int launch_fwd_sm100(const TcGeom& g, __nv_bfloat16* o, float* lse, cudaStream_t st, const SplitKV* split = nullptr);
 // O = sum_t exp(LSE_t - LSE) O_t, LSE = log sum_t exp(LSE_t) over num_parts
 // partials laid out as SplitKV's; o: bf16 (out_f32 = 0) or fp32 [B, Nq, Hq, D].

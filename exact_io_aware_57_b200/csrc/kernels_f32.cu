@@ -18,18 +18,21 @@ ATTN_DEVINL float warp_sum(float x) {
 }
 
 // Sequence geometry of one (batch or packed sequence) index z.
+// ok is false for a packed sequence with invalid offsets (reported in the
+// status word); the kernels then leave before touching any row.
 struct Seq {
   int b, q0, nq, k0, nk;
+  bool ok;
 };
 
 ATTN_DEVINL Seq seq_of(const F32Params& p, int z) {
   Seq s;
+  s.ok = true;
   if (p.cu_q) {
     s.b = 0;
-    s.q0 = p.cu_q[z];
-    s.nq = p.cu_q[z + 1] - s.q0;
-    s.k0 = p.cu_k[z];
-    s.nk = p.cu_k[z + 1] - s.k0;
+    s.ok = packed_seq(p.cu_q, z, p.Nq, p.max_nq, p.status, s.q0, s.nq) &&
+           packed_seq(p.cu_k, z, p.Nk, p.max_nk, p.status, s.k0, s.nk);
+    if (!s.ok) s.nq = s.nk = 0;
   } else {
     s.b = z;
     s.q0 = 0;
@@ -230,12 +233,14 @@ F32Params folded(const F32Params& in) {
   F32Params p = in;
   p.win_l = win_left(in.window_left);
   p.win_r = win_right(in.causal, in.window_right);
+  p.status = device_status_ptr();
   return p;
 }
 }  // namespace
 
 int launch_fwd_f32(const F32Params& in, int num_z, int max_nq, cudaStream_t st) {
   const F32Params p = folded(in);
+  if (!p.status) return ATTN_ERR_CUDA;
   dim3 grid((max_nq + 3) / 4, p.Hq, num_z);
   if (p.D == 64)
     fwd_f32_kernel<64><<<grid, 128, 0, st>>>(p);
@@ -263,6 +268,7 @@ template int launch_rowdot<__nv_bfloat16>(const __nv_bfloat16*, const __nv_bfloa
 int launch_bwd_f32(const F32Params& in, const float* dout, const float* Drow, float* dq, float* dk, float* dv,
                    int num_z, int max_nq, int max_nk, cudaStream_t st) {
   const F32Params p = folded(in);
+  if (!p.status) return ATTN_ERR_CUDA;
   dim3 gq((max_nq + 3) / 4, p.Hq, num_z), gk((max_nk + 3) / 4, p.Hkv, num_z);
   if (p.D == 64) {
     bwd_dq_f32_kernel<64><<<gq, 128, 0, st>>>(p, dout, Drow, dq);

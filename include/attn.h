@@ -188,6 +188,25 @@ int attn_merge_partials(const float* o_parts, const float* lse_parts, int num_pa
                         float* lse, int batch, int h_q, int n_q, int d, int out_dtype, void* stream);
 
 /*
+ * Partial forward over one block of keys: the exact attention of every query
+ * row over the keys given here only, left unmerged for attn_merge_partials --
+ * o_part: DEVICE fp32 [batch, n_q, h_q, d], O_t normalised over this block;
+ * lse_part: DEVICE fp32 [batch, h_q, n_q], LSE_t over this block (-inf, with
+ * O_t = 0, for a row that sees none of its keys).  Causal masking aligns the
+ * block bottom-right (key j visible from row i iff j <= i + n_k - n_q), which
+ * for n_q == n_k is the diagonal block of a sequence cut into equal chunks.
+ * This is the per-shard step when the keys of a sequence are spread over
+ * devices: each device attends to the key blocks it holds or receives and the
+ * partials merge exactly ("Softmax does not need the matrix", "Carry the
+ * Normalizer": the carried state resumes the softmax over the next block).
+ * bf16 inputs only (ATTN_ERR_UNSUPPORTED for fp32); no bias.  Otherwise as
+ * attn_fwd.
+ */
+int attn_fwd_partial(const void* q, const void* k, const void* v, float* o_part, float* lse_part,
+                     int batch, int h_q, int h_kv, int n_q, int n_k, int d, float scale, int causal,
+                     int dtype, void* stream);
+
+/*
  * attn_bwd without a workspace argument, for callers that cannot allocate
  * device memory when they run the backward (code inside a framework that owns
  * all device memory, or latency-critical loops that cannot afford cudaMalloc's
@@ -200,8 +219,10 @@ int attn_merge_partials(const float* o_parts, const float* lse_parts, int num_pa
  * allocated.  Returns ATTN_ERR_WORKSPACE when attn_bwd_workspace_size(batch,
  * h_q, n_q, d) exceeds ATTN_NOALLOC_SCRATCH_BYTES.  All calls on a device share
  * the array: calls that overlap on the GPU race.  The first call on a device
- * looks up the array's address with that device current; make it before any
- * stream capture.
+ * looks up the array's address with that device current and keeps it for the
+ * life of the process; make it before any stream capture.  A device reset
+ * (cudaDeviceReset) after that first call is not supported: the array may then
+ * sit at another address.
  */
 #define ATTN_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
 int attn_bwd_noalloc(const void* q, const void* k, const void* v, const float* bias,
@@ -216,9 +237,12 @@ int attn_bwd_noalloc(const void* q, const void* k, const void* v, const float* b
  * arrays of num_seqs + 1 non-decreasing prefix offsets starting at 0; sequence z
  * owns rows cu[z] .. cu[z+1]-1.  max_seqlen_q / max_seqlen_k bound the lengths
  * (they size the launch).  Causal masking applies inside each sequence.  No bias.
- * The offsets live in device memory and are not read on the host: offsets that
- * decrease, exceed the totals or a length above max_seqlen are the caller's
- * error, and the results are then undefined.
+ * The offsets live in device memory and are not read on the host; the kernels
+ * check them before any access: a sequence whose offsets are negative,
+ * decrease, exceed total_q / total_k, or give a length above max_seqlen_q /
+ * max_seqlen_k is neither read nor written, and ATTN_ERR_INVALID is raised in
+ * the device status word (attn_device_status); the other sequences are
+ * computed, and that sequence's outputs are left as they were.
  */
 int attn_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
                     const int* cu_seqlens_q, const int* cu_seqlens_k, int num_seqs,
@@ -242,8 +266,10 @@ const char* attn_strerror(int code);
 
 /*
  * Synchronises `stream`, then returns and clears the device status word of the
- * current device: ATTN_OK, or ATTN_ERR_TIMEOUT if a kernel launched since the
- * last call abandoned a bounded wait (its outputs are then undefined).
+ * current device: ATTN_OK; ATTN_ERR_TIMEOUT if a kernel launched since the
+ * last call abandoned a bounded wait (its outputs are then undefined); or
+ * ATTN_ERR_INVALID if a packed-sequence kernel met invalid offsets (that
+ * sequence was skipped).
  */
 int attn_device_status(void* stream);
 

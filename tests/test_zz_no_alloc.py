@@ -39,23 +39,47 @@ def _case(B, Hq, Hkv, N, d, seed):
     return q, k, v, o, lse, do
 
 
-def test_noalloc_matches_workspace_backward_twice():
+def _free_bytes():
+    free, _ = torch.cuda.mem_get_info()
+    return free
+
+
+def test_noalloc_matches_workspace_backward_twice(orc):
     from exact_io_aware_57_b200 import attn
 
     lib = attn.lib()
+    # warm-up: the first call on a device looks up the array (and may load the
+    # module that holds it); the calls measured below must allocate nothing
+    w = _case(1, 2, 2, 130, 64, 4)
+    wout = [torch.empty_like(w[0]), torch.empty_like(w[1]), torch.empty_like(w[2])]
+    assert _noalloc(lib, (*w, *wout), True, 0.125) == 0
+    torch.cuda.synchronize()
+    assert attn.attn_device_status() == 0
     # a larger call first, then a smaller one that reuses the same scratch
     for (B, Hq, Hkv, N, d, seed) in ((2, 4, 2, 777, 128, 5), (1, 2, 1, 200, 64, 6)):
         q, k, v, o, lse, do = _case(B, Hq, Hkv, N, d, seed)
         scale = 1.0 / math.sqrt(d)
         ref = attn.attn_bwd(q, k, v, o, lse, do, causal=True)
         out = [torch.full_like(q, float("nan")), torch.full_like(k, float("nan")), torch.full_like(v, float("nan"))]
+        torch.cuda.synchronize()
+        held, free0 = torch.cuda.memory_allocated(), _free_bytes()
         rc = _noalloc(lib, (q, k, v, o, lse, do, *out), True, scale)
         assert rc == 0, lib.attn_strerror(rc)
         torch.cuda.synchronize()
         assert attn.attn_device_status() == 0
+        # nothing was allocated: neither through torch nor behind its back
+        assert torch.cuda.memory_allocated() == held
+        assert _free_bytes() == free0
         for name, a, r in zip(("dq", "dk", "dv"), out, ref):
             e = rel_fro(a.cpu().double().numpy(), r.cpu().double().numpy())
             assert e <= TOL_GRAD_BF16, f"{name}: rel Frobenius {e:.3e}"
+        if seed == 6:
+            # the second call also stands on its own against the fp64 oracle
+            inp = synth.make_dense(B, Hq, Hkv, N, N, d, seed=seed)
+            dq_r, dk_r, dv_r = orc.bwd(inp.q, inp.k, inp.v, inp.dout, causal=True)
+            for name, a, r in zip(("dq", "dk", "dv"), out, (dq_r, dk_r, dv_r)):
+                e = rel_fro(a.cpu().double().numpy(), r)
+                assert e <= TOL_GRAD_BF16, f"{name} vs oracle: rel Frobenius {e:.3e}"
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch():
