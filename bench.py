@@ -51,7 +51,7 @@ def parse_args(argv=None):
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end measurement")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip timing the CPU oracle")
-    ap.add_argument("--workload", default="c3", choices=["c1", "c2", "c3", "c4", "c5a", "c5b", "kv1"],
+    ap.add_argument("--workload", default="c3", choices=["c1", "c2", "c3", "c3fp8", "c4", "c5a", "c5b", "kv1"],
                     help="c3 (default) is the headline causal fwd+bwd workload; the others are reported too")
     ap.add_argument("--batch", type=int, default=None, help="override the batch (profiling a smaller case)")
     ap.add_argument("--heads", type=int, default=None, help="override the head count (profiling a smaller case)")
@@ -154,7 +154,7 @@ def recorded_naive_ratio():
             k, v = line.split(":", 1)
             kv[k.strip()] = v.strip()
     csrc = ROOT / "exact_io_aware_57_b200" / "csrc"
-    if (kv.get("fwd_source_sha256_16") != source_digest(csrc / "fwd_sm100.cu")
+    if (kv.get("fwd_source_sha256_16") != source_digest(csrc / "fwd_pp_sm100.cu")
             or kv.get("naive_source_sha256_16") != source_digest(csrc / "naive.cu")):
         return None
     try:
@@ -302,6 +302,11 @@ def make_job(w, args, dev, rank):
                          dv=torch.empty_like(j.dev["v"]))
             ws = torch.empty(attn.attn_bwd_workspace_size(w.batch, w.h_q, w.n, w.d), device=dev, dtype=torch.uint8)
 
+        if w.fp8:
+            j.q8 = torch.empty(j.dev["q"].shape, device=dev, dtype=torch.uint8)
+            j.k8 = torch.empty(j.dev["k"].shape, device=dev, dtype=torch.uint8)
+            j.qs = torch.empty((w.batch, w.h_q), device=dev)
+            j.ks = torch.empty((w.batch, w.h_kv), device=dev)
         if w.splitkv:
             t = args.num_splits or attn.attn_splitkv_num_splits(w.batch, w.h_q, n_q, w.n)
             j.splits = t
@@ -310,6 +315,11 @@ def make_job(w, args, dev, rank):
 
         def make_step(d_, o_):
             def step():
+                if w.fp8:
+                    q8, qs = attn.attn_quantize_e4m3(d_["q"], x8=j.q8, scales=j.qs)
+                    k8, ks = attn.attn_quantize_e4m3(d_["k"], x8=j.k8, scales=j.ks)
+                    attn.attn_fwd_fp8(q8, qs, k8, ks, d_["v"], causal=w.causal, out=o_["o"], lse=o_["lse"])
+                    return
                 if w.splitkv:
                     attn.attn_fwd_splitkv(d_["q"], d_["k"], d_["v"], causal=w.causal, num_splits=j.splits,
                                           out=o_["o"], lse=o_["lse"], workspace=sws)
@@ -382,7 +392,7 @@ def run_e2e(job, n_steps, t0=None, t1=None):
     comp.wait_stream(up)
 
 
-def roofline_fracs(achieved, peaks, peak_kind, clk):
+def roofline_fracs(achieved, peaks, peak_kind, clk, fp8_half=False):
     """Fractions of one kernel's TFLOP/s against the peaks: the measured bf16
     burst figure (a kernel that ran at full clock), the measured sustained one
     (a kernel under the power cap), and NVIDIA's dense bf16 spec (the figure
@@ -392,11 +402,17 @@ def roofline_fracs(achieved, peaks, peak_kind, clk):
     sustained = float(peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"]))
     sm, smax = clk.get("sm_mhz"), clk.get("sm_max_mhz")
     capped = "sw_power_cap" in clk.get("reasons", []) or (sm and smax and sm < 0.9 * smax)
+    # FP8 forward: half of the FLOPs (S) at the e4m3 rate, twice bf16's (the nominal
+    # ratio), the other half (P V) at bf16: a FLOP-weighted peak of 4/3 of bf16's
+    mix = 4.0 / 3.0 if fp8_half else 1.0
+    burst, sustained = burst * mix, sustained * mix
+    spec = SPEC_BF16_TFLOPS * mix
     peak = sustained if capped else burst
-    return {"peak": peak, "peak_kind": f"bf16 dense, {'sustained' if capped else 'burst'}, {peak_kind}"
-                                       f" (chosen from the sampled clocks)",
+    kind = "bf16 dense" if not fp8_half else "e4m3 (S) + bf16 (P V) dense, 4/3 of bf16"
+    return {"peak": round(peak, 2), "peak_kind": f"{kind}, {'sustained' if capped else 'burst'}, {peak_kind}"
+                                                 f" (chosen from the sampled clocks)",
             "frac": round(achieved / peak, 4), "frac_of_burst": round(achieved / burst, 4),
-            "frac_of_sustained": round(achieved / sustained, 4), "frac_of_spec": round(achieved / SPEC_BF16_TFLOPS, 4)}
+            "frac_of_sustained": round(achieved / sustained, 4), "frac_of_spec": round(achieved / spec, 4)}
 
 
 def run_ours(args):
@@ -496,14 +512,14 @@ def run_ours(args):
         roofline = {"kernel": "bwd_main_kernel (tensor-core backward)" if w.backward
                     else "fwd_pp_kernel (tensor-core forward)",
                     "bound": "tensor", "achieved": round(achieved, 2), "unit": "TFLOP/s",
-                    **roofline_fracs(achieved, peaks, peak_kind, clk),
+                    **roofline_fracs(achieved, peaks, peak_kind, clk, fp8_half=w.fp8),
                     "traffic": recorded_traffic() if (w.backward and headline) else None,
                     "algorithmic_flops_per_launch": kern_flops, "avg_launch_ms": round(kern_ms, 4),
                     "target": "north-star targets are fractions of the dense bf16 spec peak (2250 TFLOP/s): "
                               "forward >= 0.60, forward+backward >= 0.45"}
         fwd_achieved = f_fwd / (fwd_ms * 1e-3) / 1e12
         fwd_roof = {"kernel": "fwd_pp_kernel (tensor-core forward)", "achieved": round(fwd_achieved, 2),
-                    **roofline_fracs(fwd_achieved, peaks, peak_kind, clk)}
+                    **roofline_fracs(fwd_achieved, peaks, peak_kind, clk, fp8_half=w.fp8)}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline and args.workload == "c3":

@@ -9,7 +9,7 @@ _BINDING_NAMES = {
     "attn_fwd", "attn_bwd", "attn_bwd_workspace_size", "attn_fwd_varlen", "attn_fwd_naive",
     "attn_naive_scratch_size", "attn_device_status", "attn_launch_count", "AttnError",
     "attn_fwd_splitkv", "attn_splitkv_num_splits", "attn_splitkv_workspace_size", "attn_merge_partials", "attn_bwd_varlen", "attn_fwd_dv",
-    "attn_fwd_partial",
+    "attn_fwd_partial", "attn_bwd_dv", "attn_quantize_e4m3", "attn_fwd_fp8",
 }
 
 

@@ -41,12 +41,16 @@ EXPORTS = {
     "attn_bwd_varlen": (_I, [_VP, _VP, _VP, _VP, _FP, _VP, _VP, _VP, _VP, _IP, _IP, _I, _I, _I, _I, _I, _I, _I, _I,
                              _F, _I, _VP, _SZ, _I, _VP]),
     "attn_fwd_dv": (_I, [_VP, _VP, _VP, _VP, _FP, _I, _I, _I, _I, _I, _I, _I, _F, _I, _I, _VP]),
+    "attn_bwd_dv": (_I, [_VP, _VP, _VP, _VP, _FP, _VP, _VP, _VP, _VP, _VP, _SZ, _I, _I, _I, _I, _I, _I, _I, _F,
+                         _I, _I, _VP]),
     "attn_selftest_wait_timeout": (_I, [ctypes.c_longlong, _VP]),
     "attn_splitkv_num_splits": (_I, [_I, _I, _I, _I]),
     "attn_splitkv_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
     "attn_fwd_splitkv": (_I, [_VP, _VP, _VP, _VP, _FP, _I, _I, _I, _I, _I, _I, _F, _I, _I, _VP, _SZ, _I, _VP]),
     "attn_merge_partials": (_I, [_FP, _FP, _I, _VP, _FP, _I, _I, _I, _I, _I, _VP]),
     "attn_fwd_partial": (_I, [_VP, _VP, _VP, _FP, _FP, _I, _I, _I, _I, _I, _I, _F, _I, _I, _VP]),
+    "attn_quantize_e4m3": (_I, [_VP, _VP, _FP, _I, _I, _I, _I, _VP]),
+    "attn_fwd_fp8": (_I, [_VP, _FP, _VP, _FP, _VP, _VP, _FP, _I, _I, _I, _I, _I, _I, _F, _I, _VP]),
     "attn_bwd_workspace_size": (_SZ, [_I, _I, _I, _I]),
     "attn_bwd": (_I, [_VP, _VP, _VP, _FP, _LL, _VP, _FP, _VP, _VP, _VP, _VP, _VP, _SZ, _I, _I, _I, _I, _I,
                       _I, _F, _I, _I, _VP]),
@@ -184,6 +188,24 @@ def attn_fwd_dv(q, k, v, causal=False, scale=None, out=None, lse=None, stream=No
     return o, lse
 
 
+def attn_bwd_dv(q, k, v, o, lse, dout, causal=False, scale=None, workspace=None, dq=None, dk=None, dv=None,
+                stream=None):
+    """Backward of attn_fwd_dv: q/k/dq/dk width d, v/o/dout/dv width d_v."""
+    B, Nq, Hq, d = q.shape
+    Nk, Hkv, d_v = k.shape[1], k.shape[2], v.shape[3]
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    if workspace is None:
+        workspace = torch.empty(attn_bwd_workspace_size(B, Hq, Nq, d), device=q.device, dtype=torch.uint8)
+    _check(_lib.attn_bwd_dv(_dev(q, "q"), _dev(k, "k"), _dev(v, "v"), _dev(o, "o"), _dev(lse, "lse"),
+                            _dev(dout, "dout"), _dev(dq, "dq"), _dev(dk, "dk"), _dev(dv, "dv"),
+                            _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(), B, Hq, Hkv,
+                            Nq, Nk, d, d_v, scale, int(bool(causal)), _dtype_code(q), _stream(stream)))
+    return dq, dk, dv
+
+
 def attn_selftest_wait_timeout(limit_cycles=1_000_000, stream=None) -> None:
     """Launch the bounded-wait self-test (a wait that gives up after limit_cycles)."""
     _check(_lib.attn_selftest_wait_timeout(int(limit_cycles), _stream(stream)))
@@ -231,6 +253,35 @@ def attn_fwd_partial(q, k, v, causal=False, scale=None, o_part=None, lse_part=No
                                  _dev(lse_part, "lse_part"), B, Hq, Hkv, Nq, Nk, d, scale, int(bool(causal)),
                                  _dtype_code(q), _stream(stream)))
     return o_part, lse_part
+
+
+def attn_quantize_e4m3(x, x8=None, scales=None, stream=None):
+    """Per-(batch, head) e4m3 quantisation of x bf16 [B,N,H,d]: returns x8 (uint8
+    e4m3 bytes, same layout) and scales fp32 [B,H] (amax / 448)."""
+    if x.dtype != torch.bfloat16:
+        raise AttnError("x must be bf16")
+    B, N, H, d = x.shape
+    x8 = torch.empty(x.shape, device=x.device, dtype=torch.uint8) if x8 is None else x8
+    scales = torch.empty((B, H), device=x.device, dtype=torch.float32) if scales is None else scales
+    _check(_lib.attn_quantize_e4m3(_dev(x, "x"), _dev(x8, "x8"), _dev(scales, "scales"), B, N, H, d,
+                                   _stream(stream)))
+    return x8, scales
+
+
+def attn_fwd_fp8(q8, q_scales, k8, k_scales, v, causal=False, scale=None, out=None, lse=None, stream=None):
+    """Forward with S = Q8 K8^T on e4m3 tensor cores (see attn_quantize_e4m3), P V in
+    bf16: o bf16 [B,Nq,Hq,d], lse fp32 [B,Hq,Nq].  d = 128."""
+    B, Nq, Hq, d = q8.shape
+    Nk, Hkv = k8.shape[1], k8.shape[2]
+    if v.dtype != torch.bfloat16:
+        raise AttnError("v must be bf16")
+    scale = 1.0 / math.sqrt(d) if scale is None else float(scale)
+    o = torch.empty((B, Nq, Hq, d), device=v.device, dtype=torch.bfloat16) if out is None else out
+    lse = torch.empty((B, Hq, Nq), device=v.device, dtype=torch.float32) if lse is None else lse
+    _check(_lib.attn_fwd_fp8(_dev(q8, "q8"), _dev(q_scales, "q_scales"), _dev(k8, "k8"), _dev(k_scales, "k_scales"),
+                             _dev(v, "v"), _dev(o, "o"), _dev(lse, "lse"), B, Hq, Hkv, Nq, Nk, d, scale,
+                             int(bool(causal)), _stream(stream)))
+    return o, lse
 
 
 def attn_merge_partials(o_parts, lse_parts, out=None, lse=None, out_dtype=torch.bfloat16, stream=None):

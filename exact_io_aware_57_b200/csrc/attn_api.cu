@@ -204,7 +204,7 @@ int bwd_impl(const void* q, const void* k, const void* v, const float* bias, lon
              void* workspace, size_t workspace_bytes, int batch, int h_q, int h_kv, int n_q, int n_k, int d,
              float scale, int causal, int window_left, int window_right, int dtype, void* stream,
              const int* cu_q = nullptr, const int* cu_k = nullptr, int num_seqs = 0, int max_nq = 0,
-             int max_nk = 0) {
+             int max_nk = 0, int d_v = 0) {
   // packed sequences: batch 1 of n_q / n_k total rows, cu_q / cu_k prefix offsets
   int rc = check_common(batch, h_q, h_kv, n_q, n_k, d, dtype);
   if (rc) return rc;
@@ -275,6 +275,7 @@ int bwd_impl(const void* q, const void* k, const void* v, const float* bias, lon
   g.num_seqs = num_seqs;
   g.max_nq = max_nq;
   g.max_nk = max_nk;
+  g.Dv = d_v;
   return launch_bwd_sm100(g, static_cast<const __nv_bfloat16*>(o), lse, static_cast<const __nv_bfloat16*>(dout),
                           static_cast<__nv_bfloat16*>(dq), static_cast<__nv_bfloat16*>(dk),
                           static_cast<__nv_bfloat16*>(dv), dq_acc, Drow, st);
@@ -320,6 +321,16 @@ int attn_bwd_varlen(const void* q, const void* k, const void* v, const void* o, 
   return bwd_impl(q, k, v, nullptr, 0, nullptr, o, lse, dout, dq, dk, dv, workspace, workspace_bytes, 1, h_q, h_kv,
                   total_q, total_k, d, scale, causal, -1, -1, dtype, stream, cu_seqlens_q, cu_seqlens_k, num_seqs,
                   max_seqlen_q, max_seqlen_k);
+}
+
+int attn_bwd_dv(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+                void* dq, void* dk, void* dv, void* workspace, size_t workspace_bytes, int batch, int h_q, int h_kv,
+                int n_q, int n_k, int d, int d_v, float scale, int causal, int dtype, void* stream) {
+  if (d_v != 64 && d_v != 128) return ATTN_ERR_UNSUPPORTED;
+  if (d_v != d && dtype != ATTN_BF16) return ATTN_ERR_UNSUPPORTED;
+  return bwd_impl(q, k, v, nullptr, 0, nullptr, o, lse, dout, dq, dk, dv, workspace, workspace_bytes, batch, h_q,
+                  h_kv, n_q, n_k, d, scale, causal, -1, -1, dtype, stream, nullptr, nullptr, 0, 0, 0,
+                  d_v == d ? 0 : d_v);
 }
 
 int attn_fwd_dv(const void* q, const void* k, const void* v, void* o, float* lse, int batch, int h_q, int h_kv,
@@ -443,6 +454,41 @@ int attn_fwd_partial(const void* q, const void* k, const void* v, float* o_part,
   sp.o_part = o_part;
   sp.lse_part = lse_part;
   return launch_fwd_sm100(g, nullptr, nullptr, static_cast<cudaStream_t>(stream), &sp);
+}
+
+int attn_quantize_e4m3(const void* x, void* x8, float* scales, int batch, int n, int heads, int d, void* stream) {
+  if (!x || !x8 || !scales || batch <= 0 || n <= 0 || heads <= 0) return ATTN_ERR_INVALID;
+  if (d != 64 && d != 128) return ATTN_ERR_UNSUPPORTED;
+  if ((long long)batch * n > (1ll << 31) - 1 || batch > 65535 || heads > 65535) return ATTN_ERR_UNSUPPORTED;
+  if (!aligned16(x) || !aligned16(x8)) return ATTN_ERR_INVALID;
+  if (!supported_device()) return ATTN_ERR_UNSUPPORTED;
+  return launch_quantize_e4m3(static_cast<const __nv_bfloat16*>(x), static_cast<uint8_t*>(x8), scales, batch, n,
+                              heads, d, static_cast<cudaStream_t>(stream));
+}
+
+int attn_fwd_fp8(const void* q8, const float* q_scales, const void* k8, const float* k_scales, const void* v,
+                 void* o, float* lse, int batch, int h_q, int h_kv, int n_q, int n_k, int d, float scale,
+                 int causal, void* stream) {
+  int rc = check_common(batch, h_q, h_kv, n_q, n_k, d, ATTN_BF16);
+  if (rc) return rc;
+  if (d != 128 || !(scale > 0.f)) return ATTN_ERR_UNSUPPORTED;
+  if (!q8 || !q_scales || !k8 || !k_scales || !v || !o || !lse) return ATTN_ERR_INVALID;
+  if (!aligned16(q8) || !aligned16(k8) || !aligned16(v) || !aligned16(o)) return ATTN_ERR_INVALID;
+  if (!supported_device()) return ATTN_ERR_UNSUPPORTED;
+  TcGeom g{};
+  g.q = q8;
+  g.k = k8;
+  g.v = v;
+  g.B = batch;
+  g.Hq = h_q;
+  g.Hkv = h_kv;
+  g.Nq = n_q;
+  g.Nk = n_k;
+  g.D = d;
+  g.causal = causal != 0;
+  g.scale = scale;
+  return launch_fwd_fp8(g, q8, q_scales, k8, k_scales, static_cast<__nv_bfloat16*>(o), lse,
+                        static_cast<cudaStream_t>(stream));
 }
 
 int attn_merge_partials(const float* o_parts, const float* lse_parts, int num_parts, void* o, float* lse, int batch,

@@ -52,19 +52,36 @@ constexpr int NSTQ = 2;   // Q/dO stages
 constexpr int kThreads = 320;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColST = 0, kColDPT = 128, kColDV = 256;
+#ifndef ATTN_BWD_EX2_EMU_EVERY
+#define ATTN_BWD_EX2_EMU_EVERY 0
+#endif
+constexpr int kBwdEmuEvery = ATTN_BWD_EX2_EMU_EVERY;
+#ifndef ATTN_BWD_SPLIT_SDP
+#define ATTN_BWD_SPLIT_SDP 0
+#endif
+// Issue S^T and dP^T one after the other (committed apart) instead of interleaved.
+constexpr bool kSplitSdp = ATTN_BWD_SPLIT_SDP != 0;
 
-template <int D>
+// D: width of Q, K, dQ, dK; DV: width of V, O, dO, dV.  The fp32 dQ tile of a
+// step (D / 32 boxes of 128 rows x 32 columns, 16 KB each) is staged in that
+// step's Q and dO buffers (D / 64 + DV / 64 boxes) and, when D > DV, in an
+// extra buffer for the boxes they cannot hold.
+template <int D, int DV>
 struct BwdSmem {
-  static constexpr int kTileBytes = 128 * D * 2;
-  alignas(1024) uint8_t k[kTileBytes];
-  alignas(1024) uint8_t v[kTileBytes];
-  alignas(1024) uint8_t q[NSTQ][kTileBytes];
-  alignas(1024) uint8_t dout[NSTQ][kTileBytes];
+  static constexpr int kKBytes = 128 * D * 2;
+  static constexpr int kVBytes = 128 * DV * 2;
+  static constexpr int kQBoxes = D / 64, kDoBoxes = DV / 64;
+  static constexpr int kXBoxes = D / 32 > kQBoxes + kDoBoxes ? D / 32 - kQBoxes - kDoBoxes : 0;
+  alignas(1024) uint8_t k[kKBytes];
+  alignas(1024) uint8_t v[kVBytes];
+  alignas(1024) uint8_t q[NSTQ][kKBytes];
+  alignas(1024) uint8_t dout[NSTQ][kVBytes];
   alignas(1024) uint8_t ds[128 * 128 * 2];  // dS^T, [key][query] in two 64-column blocks
+  alignas(1024) uint8_t dqx[NSTQ][kXBoxes > 0 ? kXBoxes * 128 * 128 : 16];
   alignas(16) float nlse2[NSTQ][BM];        // -log2(e) * LSE of the step's query rows (-inf: no key)
   alignas(16) float drow[NSTQ][BM];         // D_i of the step's query rows
   uint64_t kv_full, q_full[NSTQ], staged[NSTQ];
-  uint64_t st_full, s_read, ds_ready, dkq_done, tmem_free, drain;
+  uint64_t st_full, dp_full, s_read, ds_ready, dkq_done, tmem_free, drain;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -142,7 +159,8 @@ ATTN_DEVINL void p_chunk(int c, const uint32_t (&sr)[32], uint32_t st_col, const
       float t = fmaf(__uint_as_float(sr[e]), scale_log2, nlv[u]);
       if constexpr (BIAS == kBiasDense) t = fmaf(__ldg(bcol + (long long)min(q0 + e, len_q - 1) * nk), kLog2e, t);
       if constexpr (BIAS == kBiasAlibi) t = fmaf(neg_slope2, fabsf(static_cast<float>(kj - q0 - e - bias_diag)), t);
-      float pe = ex2(t);
+      // unmasked tiles (every t finite): one exponential in kBwdEmuEvery on the FMA pipe
+      float pe = (!MASK && kBwdEmuEvery > 0 && e % kBwdEmuEvery == kBwdEmuEvery - 1) ? ex2_poly(t) : ex2(t);
       if constexpr (MASK) pe = (e >= vis_lo && e < vis_hi) ? pe : 0.f;
       pv[u] = pe;
     }
@@ -229,14 +247,14 @@ ATTN_DEVINL void bwd_ds_half(int grp, uint32_t st_col, uint32_t dp_col, const fl
   ds_chunk(c0 + 1, pb, db, drow, ds_row, r);
 }
 
-template <int D, int BIAS>
+template <int D, int DV, int BIAS>
 __global__ void __launch_bounds__(kThreads, 1)
     bwd_main_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                     const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
                     const __grid_constant__ CUtensorMap tm_dq, const BwdParams p) {
-  using Smem = BwdSmem<D>;
-  constexpr int KB = D / 64;
-  constexpr uint32_t kColDK = kColDV + D;
+  using Smem = BwdSmem<D, DV>;
+  constexpr int KB = D / 64, KBV = DV / 64;
+  constexpr uint32_t kColDK = kColDV + DV;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   Smem& s = *reinterpret_cast<Smem*>(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -274,6 +292,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&s.staged[i], 8);   // the eight elementwise warps, dQ tile staged
     }
     mbar_init(&s.st_full, 1);
+    mbar_init(&s.dp_full, 1);
     mbar_init(&s.s_read, 4);
     mbar_init(&s.ds_ready, 8);
     mbar_init(&s.dkq_done, 1);
@@ -288,7 +307,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = s.tmem_base;
   const Abort ab{&s.abort_flag, p.status, p.wait_limit};
 
-  constexpr int kBoxes = D / 64;  // 16 KB fp32 dQ boxes (128 rows x 32 columns) per Q or dO buffer
+  // staging place of fp32 dQ box c (columns 32c .. 32c + 31) of stage st
+  auto dq_box = [&](int st, int c) -> uint8_t* {
+    if (c < Smem::kQBoxes) return s.q[st] + c * (128 * 128);
+    if (c < Smem::kQBoxes + Smem::kDoBoxes) return s.dout[st] + (c - Smem::kQBoxes) * (128 * 128);
+    return s.dqx[st] + (c - Smem::kQBoxes - Smem::kDoBoxes) * (128 * 128);
+  };
   if (warp == 0) {
     // ===================================================== producer
     // Stage st of step s held the dQ tile of step s - NSTQ: before reloading
@@ -303,8 +327,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int i0 = (i_first + t % per_head) * BM;
 #pragma unroll
         for (int c = 0; c < D / 32; ++c)
-          tma_reduce_add_4d(&tm_dq, (c < kBoxes ? s.q[st] : s.dout[st]) + (c % kBoxes) * (128 * 128), c * 32, h,
-                            q_off + i0, b);
+          tma_reduce_add_4d(&tm_dq, dq_box(st, c), c * 32, h, q_off + i0, b);
         bulk_commit();
         bulk_wait_read0();
       }
@@ -319,12 +342,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_prefetch_desc(&tm_do);
       tma_prefetch_desc(&tm_dq);
       if (n_steps > 0) {
-        mbar_expect_tx(&s.kv_full, 2 * Smem::kTileBytes);
+        mbar_expect_tx(&s.kv_full, Smem::kKBytes + Smem::kVBytes);
 #pragma unroll
-        for (int kb = 0; kb < KB; ++kb) {
-          tma_load_4d(s.k + kb * BN * 128, &tm_k, &s.kv_full, kb * 64, hk, k_off + n0, b);
-          tma_load_4d(s.v + kb * BN * 128, &tm_v, &s.kv_full, kb * 64, hk, k_off + n0, b);
-        }
+        for (int kb = 0; kb < KB; ++kb) tma_load_4d(s.k + kb * BN * 128, &tm_k, &s.kv_full, kb * 64, hk, k_off + n0, b);
+#pragma unroll
+        for (int kb = 0; kb < KBV; ++kb) tma_load_4d(s.v + kb * BN * 128, &tm_v, &s.kv_full, kb * 64, hk, k_off + n0, b);
       }
     }
     bool ok = true;
@@ -349,12 +371,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (step >= NSTQ && !(ok = reduce_step(step - NSTQ))) break;
       if (lane == 0) {
-        mbar_expect_tx(&s.q_full[st], 2 * Smem::kTileBytes);
+        mbar_expect_tx(&s.q_full[st], Smem::kKBytes + Smem::kVBytes);
 #pragma unroll
-        for (int kb = 0; kb < KB; ++kb) {
+        for (int kb = 0; kb < KB; ++kb)
           tma_load_4d(s.q[st] + kb * BM * 128, &tm_q, &s.q_full[st], kb * 64, h, q_off + i0, b);
+#pragma unroll
+        for (int kb = 0; kb < KBV; ++kb)
           tma_load_4d(s.dout[st] + kb * BM * 128, &tm_do, &s.q_full[st], kb * 64, h, q_off + i0, b);
-        }
       }
 #pragma unroll
       for (int e = 0; e < BM / 32; ++e) {
@@ -378,7 +401,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ===================================================== MMA issuer
     if (lane == 0 && n_steps > 0) {
       constexpr uint32_t idesc_s = idesc_bf16(BN, BM, 0, 0);    // K_j / V_j (K-major) x Q_i / dO_i (K-major)
-      constexpr uint32_t idesc_kv = idesc_bf16(BN, D, 0, 1);    // P^T, dS^T (K-major) x dO_i / Q_i (MN-major)
+      constexpr uint32_t idesc_dv = idesc_bf16(BN, DV, 0, 1);   // P^T (K-major) x dO_i (MN-major)
+      constexpr uint32_t idesc_kv = idesc_bf16(BN, D, 0, 1);    // dS^T (K-major) x Q_i (MN-major)
       constexpr uint32_t idesc_dq = idesc_bf16(BM, D, 1, 1);    // dS (MN-major) x K_j (MN-major)
       const uint32_t k_addr = smem_u32(s.k), v_addr = smem_u32(s.v), ds_addr = smem_u32(s.ds);
       bool ok = mbar_wait(&s.kv_full, 0, ab);
@@ -391,22 +415,47 @@ __global__ void __launch_bounds__(kThreads, 1)
         // earlier by this thread: tcgen05.mma executes in issue order) and
         // dP^T = V_j dO_i^T, round-robin.  dP^T goes where dQ of the previous
         // step was: the first S^T MMA is issued before waiting for it to leave.
-        mma_ss(tmem + kColST, sdesc_sw128(k_addr, 16, 1024), sdesc_sw128(q_addr, 16, 1024), idesc_s, false);
-        if (step > 0 && !mbar_wait(&s.tmem_free, (step - 1) & 1, ab)) break;
-        tc_fence_after();
+        if constexpr (kSplitSdp) {
+          // S^T alone first (the elementwise groups start P^T on it), then
+          // dP^T once the previous dQ has left TMEM
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
-          const uint32_t off1 = ((kk + 1) >> 2) * (128 * 128) + ((kk + 1) & 3) * 32;
-          mma_ss(tmem + kColDPT, sdesc_sw128(v_addr + off, 16, 1024), sdesc_sw128(do_addr + off, 16, 1024),
-                 idesc_s, kk > 0);
-          if (kk + 1 < D / 16)
-            mma_ss(tmem + kColST, sdesc_sw128(k_addr + off1, 16, 1024), sdesc_sw128(q_addr + off1, 16, 1024),
-                   idesc_s, true);
+          for (int kk = 0; kk < D / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+            mma_ss(tmem + kColST, sdesc_sw128(k_addr + off, 16, 1024), sdesc_sw128(q_addr + off, 16, 1024), idesc_s,
+                   kk > 0);
+          }
+          // its completion also implies that the previous step's MMAs, the last
+          // readers of the dS^T tile, are done
+          mma_commit(&s.st_full);
+          if (step > 0 && !mbar_wait(&s.tmem_free, (step - 1) & 1, ab)) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < DV / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+            mma_ss(tmem + kColDPT, sdesc_sw128(v_addr + off, 16, 1024), sdesc_sw128(do_addr + off, 16, 1024),
+                   idesc_s, kk > 0);
+          }
+          mma_commit(&s.dp_full);
+        } else {
+          mma_ss(tmem + kColST, sdesc_sw128(k_addr, 16, 1024), sdesc_sw128(q_addr, 16, 1024), idesc_s, false);
+          if (step > 0 && !mbar_wait(&s.tmem_free, (step - 1) & 1, ab)) break;
+          tc_fence_after();
+#pragma unroll
+          for (int kk = 0; kk < (D > DV ? D : DV) / 16; ++kk) {
+            const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+            const uint32_t off1 = ((kk + 1) >> 2) * (128 * 128) + ((kk + 1) & 3) * 32;
+            if (kk < DV / 16)
+              mma_ss(tmem + kColDPT, sdesc_sw128(v_addr + off, 16, 1024), sdesc_sw128(do_addr + off, 16, 1024),
+                     idesc_s, kk > 0);
+            if (kk + 1 < D / 16)
+              mma_ss(tmem + kColST, sdesc_sw128(k_addr + off1, 16, 1024), sdesc_sw128(q_addr + off1, 16, 1024),
+                     idesc_s, true);
+          }
+          // its completion also implies that the previous step's MMAs, the last
+          // readers of the dS^T tile, are done
+          mma_commit(&s.st_full);
+          mma_commit(&s.dp_full);
         }
-        // its completion also implies that the previous step's MMAs, the last
-        // readers of the dS^T tile, are done
-        mma_commit(&s.st_full);
         if (!mbar_wait(&s.ds_ready, step & 1, ab)) break;
         tc_fence_after();
         // dV += P^T dO_i (P^T from TMEM), dK += dS^T Q_i and dQ_i = dS K_j (the
@@ -414,7 +463,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk) {
           const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
-          mma_ts(tmem + kColDV, tmem + kColST + kk * 8, sdesc_sw128(do_addr + kk * 2048, BM * 128, 1024), idesc_kv,
+          mma_ts(tmem + kColDV, tmem + kColST + kk * 8, sdesc_sw128(do_addr + kk * 2048, BM * 128, 1024), idesc_dv,
                  (step > 0 || kk > 0));
           mma_ss(tmem + kColDK, sdesc_sw128(ds_addr + off, 16, 1024), sdesc_sw128(q_addr + kk * 2048, BM * 128, 1024),
                  idesc_kv, (step > 0 || kk > 0));
@@ -462,6 +511,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                                      neg_slope2, p.Nk, i0, len_q, kj, len_k, 0, 0, diag);
       if (!ok) break;
       tmem_wait_st();
+      // dP^T of this step (committed with S^T unless the two are split)
+      ok = __all_sync(0xffffffffu, mbar_wait(&s.dp_full, step & 1, ab));
+      if (!ok) break;
+      tc_fence_after();
       bwd_ds_half(grp, st_col, dp_col, s.drow[st], ds_row, r);
       fence_proxy_async_smem();
       tc_fence_before();
@@ -480,13 +533,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s.tmem_free);
-      // box c (columns 32c .. 32c+31, 16 KB): each buffer holds D / 64 boxes,
-      // Q_i's first, then dO_i's; 128B-swizzled like the TMA map
-      const uint32_t q_row = smem_u32(s.q[st]) + r * 128, do_row = smem_u32(s.dout[st]) + r * 128;
+      // box c (columns 32c .. 32c+31, 16 KB) at dq_box(st, c), 128B-swizzled like the TMA map
 #pragma unroll
       for (int cl = 0; cl < D / 64; ++cl) {
         const int c = grp * (D / 64) + cl;
-        const uint32_t row = (c < kBoxes ? q_row : do_row) + (c % kBoxes) * (128 * 128);
+        const uint32_t row = smem_u32(dq_box(st, c)) + r * 128;
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
           const int e = cl * 32 + 4 * u;
@@ -497,19 +548,21 @@ __global__ void __launch_bounds__(kThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&s.staged[st]);
     }
-    // ---- epilogue: dK (scaled) and dV, key row r, columns [grp D/2, grp D/2 + D/2)
-    // the MMA warp commits `drain` after its last MMA
+    // ---- epilogue: dV (columns [grp DV/2, grp DV/2 + DV/2)) and dK (scaled,
+    // columns [grp D/2, grp D/2 + D/2)) of key row r.  The MMA warp commits
+    // `drain` after its last MMA
     if (ok && n_steps > 0) ok = __all_sync(0xffffffffu, mbar_wait(&s.drain, 0, ab));
     tc_fence_after();
     if (ok) {
-      const long long row = (((long long)b * p.Nk + k_off + kj) * p.Hkv + hk) * D + grp * (D / 2);
+      const long long key = ((long long)b * p.Nk + k_off + kj) * p.Hkv + hk;
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
-        const uint32_t col0 = (half == 0 ? kColDV : kColDK) + grp * (D / 2);
+        const int W = half == 0 ? DV : D;
+        const uint32_t col0 = (half == 0 ? kColDV : kColDK) + grp * (W / 2);
         const float mul = half == 0 ? 1.f : p.scale;
-        __nv_bfloat16* dst = (half == 0 ? p.dv : p.dk) + row;
+        __nv_bfloat16* dst = (half == 0 ? p.dv : p.dk) + key * W + grp * (W / 2);
 #pragma unroll
-        for (int c = 0; c < D / 64; ++c) {
+        for (int c = 0; c < W / 64; ++c) {
           uint32_t a[32];
           if (n_steps > 0) {
             tmem_ld32(tmem + lane_off + col0 + c * 32, a);
@@ -542,25 +595,26 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-// D_i = dO_i . O_i (fp32) and zeroed dQ accumulator rows.  One warp per (b, n, h) row.
-template <int D>
+// D_i = dO_i . O_i (fp32, rows of DV) and zeroed dQ accumulator rows (D).  One
+// warp per (b, n, h) row.
+template <int D, int DV>
 __global__ void __launch_bounds__(256) bwd_pre_kernel(const __nv_bfloat16* __restrict__ o,
                                                       const __nv_bfloat16* __restrict__ dout, float* __restrict__ drow,
                                                       float* __restrict__ dq_acc, int B, int Hq, int Nq) {
-  constexpr int E = D / 32;  // bf16 per lane (2 or 4)
+  constexpr int EV = DV / 32, EQ = D / 32;  // elements per lane (2 or 4)
   const long long row = (long long)blockIdx.x * 8 + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (row >= (long long)B * Nq * Hq) return;
   float acc = 0.f;
-  const __nv_bfloat16* orow = o + row * D + lane * E;
-  const __nv_bfloat16* drw = dout + row * D + lane * E;
+  const __nv_bfloat16* orow = o + row * DV + lane * EV;
+  const __nv_bfloat16* drw = dout + row * DV + lane * EV;
 #pragma unroll
-  for (int e = 0; e < E; ++e) acc = fmaf(__bfloat162float(orow[e]), __bfloat162float(drw[e]), acc);
+  for (int e = 0; e < EV; ++e) acc = fmaf(__bfloat162float(orow[e]), __bfloat162float(drw[e]), acc);
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-  float* q = dq_acc + row * D + lane * E;
+  float* q = dq_acc + row * D + lane * EQ;
 #pragma unroll
-  for (int e = 0; e < E; ++e) q[e] = 0.f;
+  for (int e = 0; e < EQ; ++e) q[e] = 0.f;
   if (lane == 0) {
     const int h = (int)(row % Hq);
     const long long bn = row / Hq;
@@ -580,11 +634,11 @@ __global__ void __launch_bounds__(256) bwd_dq_kernel(const float* __restrict__ a
                                                pack_bf16(c.x * scale, c.y * scale), pack_bf16(c.z * scale, c.w * scale));
 }
 
-template <int D, int BIAS>
+template <int D, int DV, int BIAS>
 int launch_main_t(const TcGeom& g, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                   const CUtensorMap& mdo, const CUtensorMap& mdq, const BwdParams& p, cudaStream_t st) {
-  const size_t smem = std::max<size_t>(sizeof(BwdSmem<D>), 116 * 1024);
-  auto kern = bwd_main_kernel<D, BIAS>;
+  const size_t smem = std::max<size_t>(sizeof(BwdSmem<D, DV>), 116 * 1024);
+  auto kern = bwd_main_kernel<D, DV, BIAS>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return ATTN_ERR_CUDA;
   dim3 grid(((g.cu_q ? g.max_nk : g.Nk) + BN - 1) / BN, g.Hkv, g.cu_q ? g.num_seqs : g.B);
@@ -601,14 +655,19 @@ int launch_bwd_sm100(const TcGeom& g, const __nv_bfloat16* o, const float* lse, 
                      __nv_bfloat16* dq, __nv_bfloat16* dk, __nv_bfloat16* dv, float* dq_acc, float* Drow,
                      cudaStream_t st) {
   // packed sequences are one batch of g.Nq / g.Nk total rows
+  const int dvw = g.Dv ? g.Dv : g.D;  // width of V, O, dO, dV
   // 1) D and zeroed accumulator
   {
     const long long rows = (long long)g.B * g.Nq * g.Hq;
     const unsigned blocks = (unsigned)((rows + 7) / 8);
-    if (g.D == 64)
-      bwd_pre_kernel<64><<<blocks, 256, 0, st>>>(o, dout, Drow, dq_acc, g.B, g.Hq, g.Nq);
+    if (g.D == 64 && dvw == 64)
+      bwd_pre_kernel<64, 64><<<blocks, 256, 0, st>>>(o, dout, Drow, dq_acc, g.B, g.Hq, g.Nq);
+    else if (g.D == 128 && dvw == 128)
+      bwd_pre_kernel<128, 128><<<blocks, 256, 0, st>>>(o, dout, Drow, dq_acc, g.B, g.Hq, g.Nq);
+    else if (g.D == 128)
+      bwd_pre_kernel<128, 64><<<blocks, 256, 0, st>>>(o, dout, Drow, dq_acc, g.B, g.Hq, g.Nq);
     else
-      bwd_pre_kernel<128><<<blocks, 256, 0, st>>>(o, dout, Drow, dq_acc, g.B, g.Hq, g.Nq);
+      bwd_pre_kernel<64, 128><<<blocks, 256, 0, st>>>(o, dout, Drow, dq_acc, g.B, g.Hq, g.Nq);
     count_launch();
     if (cudaGetLastError() != cudaSuccess) return ATTN_ERR_CUDA;
   }
@@ -619,7 +678,9 @@ int launch_bwd_sm100(const TcGeom& g, const __nv_bfloat16* o, const float* lse, 
     const uint64_t dims[4] = {(uint64_t)g.D, (uint64_t)g.Hq, (uint64_t)g.Nq, (uint64_t)g.B};
     const uint64_t str[3] = {(uint64_t)g.D * 2, (uint64_t)g.Hq * g.D * 2, (uint64_t)g.Nq * g.Hq * g.D * 2};
     if (encode_tmap_bf16(&mq, g.q, 4, dims, str, box) != ATTN_OK) return ATTN_ERR_CUDA;
-    if (encode_tmap_bf16(&mdo, dout, 4, dims, str, box) != ATTN_OK) return ATTN_ERR_CUDA;
+    const uint64_t dv_dims[4] = {(uint64_t)dvw, (uint64_t)g.Hq, (uint64_t)g.Nq, (uint64_t)g.B};
+    const uint64_t dv_str[3] = {(uint64_t)dvw * 2, (uint64_t)g.Hq * dvw * 2, (uint64_t)g.Nq * g.Hq * dvw * 2};
+    if (encode_tmap_bf16(&mdo, dout, 4, dv_dims, dv_str, box) != ATTN_OK) return ATTN_ERR_CUDA;
     // fp32 accumulator: 32 floats (128 bytes) x 128 rows per box
     const uint64_t str32[3] = {(uint64_t)g.D * 4, (uint64_t)g.Hq * g.D * 4, (uint64_t)g.Nq * g.Hq * g.D * 4};
     const uint32_t box32[4] = {32, 1, 128, 1};
@@ -630,7 +691,9 @@ int launch_bwd_sm100(const TcGeom& g, const __nv_bfloat16* o, const float* lse, 
     const uint64_t dims[4] = {(uint64_t)g.D, (uint64_t)g.Hkv, (uint64_t)g.Nk, (uint64_t)g.B};
     const uint64_t str[3] = {(uint64_t)g.D * 2, (uint64_t)g.Hkv * g.D * 2, (uint64_t)g.Nk * g.Hkv * g.D * 2};
     if (encode_tmap_bf16(&mk, g.k, 4, dims, str, box) != ATTN_OK) return ATTN_ERR_CUDA;
-    if (encode_tmap_bf16(&mv, g.v, 4, dims, str, box) != ATTN_OK) return ATTN_ERR_CUDA;
+    const uint64_t dv_dims[4] = {(uint64_t)dvw, (uint64_t)g.Hkv, (uint64_t)g.Nk, (uint64_t)g.B};
+    const uint64_t dv_str[3] = {(uint64_t)dvw * 2, (uint64_t)g.Hkv * dvw * 2, (uint64_t)g.Nk * g.Hkv * dvw * 2};
+    if (encode_tmap_bf16(&mv, g.v, 4, dv_dims, dv_str, box) != ATTN_OK) return ATTN_ERR_CUDA;
   }
   BwdParams p{};
   p.lse = lse;
@@ -658,14 +721,18 @@ int launch_bwd_sm100(const TcGeom& g, const __nv_bfloat16* o, const float* lse, 
   p.wait_limit = kWaitLimitCycles;
   if (!p.status) return ATTN_ERR_CUDA;
   int rc;
-  if (g.D == 64)
-    rc = g.bias    ? launch_main_t<64, kBiasDense>(g, mq, mk, mv, mdo, mdq, p, st)
-         : g.alibi ? launch_main_t<64, kBiasAlibi>(g, mq, mk, mv, mdo, mdq, p, st)
-                   : launch_main_t<64, kBiasNone>(g, mq, mk, mv, mdo, mdq, p, st);
+  if (dvw != g.D)  // value width of its own: no bias
+    rc = (g.bias || g.alibi) ? ATTN_ERR_UNSUPPORTED
+         : g.D == 128        ? launch_main_t<128, 64, kBiasNone>(g, mq, mk, mv, mdo, mdq, p, st)
+                             : launch_main_t<64, 128, kBiasNone>(g, mq, mk, mv, mdo, mdq, p, st);
+  else if (g.D == 64)
+    rc = g.bias    ? launch_main_t<64, 64, kBiasDense>(g, mq, mk, mv, mdo, mdq, p, st)
+         : g.alibi ? launch_main_t<64, 64, kBiasAlibi>(g, mq, mk, mv, mdo, mdq, p, st)
+                   : launch_main_t<64, 64, kBiasNone>(g, mq, mk, mv, mdo, mdq, p, st);
   else
-    rc = g.bias    ? launch_main_t<128, kBiasDense>(g, mq, mk, mv, mdo, mdq, p, st)
-         : g.alibi ? launch_main_t<128, kBiasAlibi>(g, mq, mk, mv, mdo, mdq, p, st)
-                   : launch_main_t<128, kBiasNone>(g, mq, mk, mv, mdo, mdq, p, st);
+    rc = g.bias    ? launch_main_t<128, 128, kBiasDense>(g, mq, mk, mv, mdo, mdq, p, st)
+         : g.alibi ? launch_main_t<128, 128, kBiasAlibi>(g, mq, mk, mv, mdo, mdq, p, st)
+                   : launch_main_t<128, 128, kBiasNone>(g, mq, mk, mv, mdo, mdq, p, st);
   if (rc) return rc;
   // 3) dQ
   const long long n8 = (long long)g.B * g.Nq * g.Hq * g.D / 8;

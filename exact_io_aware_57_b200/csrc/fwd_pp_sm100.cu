@@ -63,14 +63,15 @@ constexpr float kRescaleThreshold = 8.f;  // log2 units: P stays <= 256
 constexpr int kEmuEvery = ATTN_EX2_EMU_EVERY;
 
 // K/V ring depth: as many stages as fit beside the two Q tiles in ~220 KB.
-template <int D, int DV>
-constexpr int kStages = (D == 128 && DV == 128) ? 2 : (D == 64 && DV == 64) ? 4 : 3;
+// QK8: Q and K held as e4m3 (one byte per element) for the FP8 forward.
+template <int D, int DV, bool QK8>
+constexpr int kStages = QK8 ? 3 : (D == 128 && DV == 128) ? 2 : (D == 64 && DV == 64) ? 4 : 3;
 
-template <int D, int DV>
+template <int D, int DV, bool QK8 = false>
 struct PPSmem {
-  static constexpr int NST = kStages<D, DV>;
-  static constexpr int kQBytes = BM * D * 2;
-  static constexpr int kKBytes = BN * D * 2;
+  static constexpr int NST = kStages<D, DV, QK8>;
+  static constexpr int kQBytes = BM * D * (QK8 ? 1 : 2);
+  static constexpr int kKBytes = BN * D * (QK8 ? 1 : 2);
   static constexpr int kVBytes = BN * DV * 2;
   alignas(1024) uint8_t q[2][kQBytes];
   alignas(1024) uint8_t k[NST][kKBytes];
@@ -110,15 +111,16 @@ ATTN_DEVINL TileRange tile_range(int mt, int len_q, int diag, int win_l, int win
 
 ATTN_DEVINL bool in_range(const TileRange& r, int j) { return r.n > 0 && j >= r.jb && j < r.jb + r.n; }
 
-template <int D, int DV, int BIAS, bool FAST, bool PARTIAL>
 // 10 warps: three of them share one SM sub-partition's 16K registers, so a
 // thread gets at most 168.
+template <int D, int DV, int BIAS, bool FAST, bool PARTIAL, bool QK8 = false>
 __global__ void __launch_bounds__(kThreads, 1)
     fwd_pp_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
-  using Smem = PPSmem<D, DV>;
+  using Smem = PPSmem<D, DV, QK8>;
   constexpr int NST = Smem::NST;
-  constexpr int KB = D / 64;  // 64-column (128-byte) blocks per Q/K row
+  constexpr int KB = D * (QK8 ? 1 : 2) / 128;  // 128-byte blocks per Q/K row
+  constexpr int kBoxCols = QK8 ? 128 : 64;     // elements in one 128-byte block
   extern __shared__ uint8_t smem_raw[];
   Smem& s = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -187,7 +189,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (rg[t].n == 0) continue;
 #pragma unroll
         for (int kb = 0; kb < KB; ++kb)
-          tma_load_4d(s.q[t] + kb * BM * 128, &tm_q, &s.q_full, kb * 64, h, q_off + m0 + t * BM, bidx);
+          tma_load_4d(s.q[t] + kb * BM * 128, &tm_q, &s.q_full, kb * kBoxCols, h, q_off + m0 + t * BM, bidx);
       }
       int issued_k = 0, issued_v = 0;
       for (int i = 0; i < n_union; ++i) {
@@ -198,7 +200,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_expect_tx(&s.k_full[st], Smem::kKBytes);
 #pragma unroll
         for (int kb = 0; kb < KB; ++kb)
-          tma_load_4d(s.k[st] + kb * BN * 128, &tm_k, &s.k_full[st], kb * 64, hk, row, bidx);
+          tma_load_4d(s.k[st] + kb * BN * 128, &tm_k, &s.k_full[st], kb * kBoxCols, hk, row, bidx);
         ++issued_k;
         if (!mbar_wait(&s.v_empty[st], ph ^ 1, ab)) break;
         mbar_expect_tx(&s.v_full[st], Smem::kVBytes);
@@ -228,11 +230,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!mbar_wait(&s.k_full[st], (i / NST) & 1, ab)) return false;
         tc_fence_after();
         const uint32_t q_addr = smem_u32(s.q[t]), k_addr = smem_u32(s.k[st]);
+        // one instruction per 32 bytes of the rows: K = 16 (bf16) or 32 (e4m3) elements
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
+        for (int kk = 0; kk < KB * 4; ++kk) {
           const uint32_t off = (kk >> 2) * (BM * 128) + (kk & 3) * 32;
-          mma_ss(tmem + t * 128, sdesc_sw128(q_addr + off, 16, 1024), sdesc_sw128(k_addr + off, 16, 1024), idesc_s,
-                 kk > 0);
+          if constexpr (QK8)
+            mma_ss_f8(tmem + t * 128, sdesc_sw128(q_addr + off, 16, 1024), sdesc_sw128(k_addr + off, 16, 1024),
+                      idesc_e4m3(BM, BN), kk > 0);
+          else
+            mma_ss(tmem + t * 128, sdesc_sw128(q_addr + off, 16, 1024), sdesc_sw128(k_addr + off, 16, 1024), idesc_s,
+                   kk > 0);
         }
         mma_commit(&s.s_full[t]);
         if (t == 1 || !in_range(rg[1], j)) mma_commit(&s.k_empty[st]);
@@ -285,6 +292,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       brow = p.bias + bidx * p.bias_bstride + ((long long)h * p.Nq + min(i, len_q - 1)) * p.Nk;
     float neg_slope2 = 0.f;  // ALiBi: B = -slope |key - (i + diag)|, in log2 units
     if constexpr (BIAS == kBiasAlibi) neg_slope2 = -__ldg(p.alibi + h) * kLog2e;
+    // log2(e) * scale, times the e4m3 scales of this (batch, head) of Q and K in the FP8 forward
+    float sc2 = p.scale_log2;
+    if constexpr (QK8) sc2 *= __ldg(p.q_scale + bidx * p.Hq + h) * __ldg(p.k_scale + bidx * p.Hkv + hk);
     float m = -INFINITY, l = 0.f;
     bool ok = true;
     for (int step = 0; step < my.n; ++step) {
@@ -298,127 +308,76 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int hi = min(len_k, i + diag + p.win_r + 1) - kbase;
       const int lo = i + diag - p.win_l - kbase;
       float alpha, m_next, rs0 = 0.f, rs1 = 0.f;
-      if constexpr (FAST) {
-        // ---- no bias, positive scale: the max may be taken on the raw scores.
-        // Pass 1 reads the scores for the row max only, 64 columns at a time;
-        // pass 2 reads them again 32 at a time (the next load in flight while
-        // the current one is exponentiated), so that few registers stay live.
-        float mx0 = -INFINITY, mx1 = -INFINITY;
+      // every score of the row in registers (one TMEM pass): x = s * scale * log2(e)
+      // (+ bias * log2(e)) in the general case; the FAST case defers the scale
+      uint32_t sr[BN];
 #pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
-          uint32_t a[32], b[32];
-          tmem_ld32(col_s + hh * 64, a);
-          tmem_ld32(col_s + hh * 64 + 32, b);
-          tmem_wait_ld();
-          reg_fence(a);
-          reg_fence(b);
-#pragma unroll
-          for (int c = 0; c < 32; ++c) {
-            float va = __uint_as_float(a[c]), vb = __uint_as_float(b[c]);
-            if (edge) {
-              const int ka = hh * 64 + c, kb = ka + 32;
-              va = (ka >= hi || ka < lo) ? -INFINITY : va;
-              vb = (kb >= hi || kb < lo) ? -INFINITY : vb;
-            }
-            mx0 = fmaxf(mx0, va);
-            mx1 = fmaxf(mx1, vb);
-          }
-        }
-        const float mx = fmaxf(mx0, mx1) * p.scale_log2;  // scale > 0: max commutes with it
-        const bool move = mx > m + kRescaleThreshold;
-        m_next = move ? mx : m;
-        alpha = move ? ex2(m - m_next) : 1.f;
-        const float neg_m = m_next == -INFINITY ? 0.f : -m_next;
-        // P over the score columns already read: 32 keys -> 16 bf16 pairs per
-        // store (P chunk c covers columns [16c, 16c + 16), scores of chunk c/2).
-        // On tiles with no hidden key one pair in kEmuEvery takes the FMA-pipe
-        // exponential instead of the MUFU one.
-        auto pass2 = [&](auto edge_c) {
-          constexpr bool EDGE = decltype(edge_c)::value;
-          uint32_t cur[32];
-          tmem_ld32(col_s, cur);
-          tmem_wait_ld();
-          reg_fence(cur);
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            uint32_t nxt[32];
-            if (c < 3) tmem_ld32(col_s + (c + 1) * 32, nxt);
-            uint32_t pk[16];
-#pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              float a0 = fmaf(__uint_as_float(cur[2 * e]), p.scale_log2, neg_m);
-              float a1 = fmaf(__uint_as_float(cur[2 * e + 1]), p.scale_log2, neg_m);
-              float p0, p1;
-              if constexpr (EDGE) {
-                const int k0 = c * 32 + 2 * e;
-                a0 = (k0 >= hi || k0 < lo) ? -INFINITY : a0;
-                a1 = (k0 + 1 >= hi || k0 + 1 < lo) ? -INFINITY : a1;
-                p0 = ex2(a0);
-                p1 = ex2(a1);
-              } else if (kEmuEvery > 0 && e % kEmuEvery == kEmuEvery - 1) {
-                p0 = ex2_poly(a0);
-                p1 = ex2_poly(a1);
-              } else {
-                p0 = ex2(a0);
-                p1 = ex2(a1);
-              }
-              rs0 += p0;
-              rs1 += p1;
-              pk[e] = pack_bf16(p0, p1);
-            }
-            tmem_st16(col_s + c * 16, pk);
-            if (c < 3) {
-              tmem_wait_ld();
-              reg_fence(nxt);
-#pragma unroll
-              for (int e = 0; e < 32; ++e) cur[e] = nxt[e];
-            }
-          }
-        };
-        if (edge)
-          pass2(std::true_type{});
-        else
-          pass2(std::false_type{});
-      } else {
-        // ---- general scores: x = s * scale * log2(e) (+ bias * log2(e)), one pass
-        uint32_t sr[BN];
-#pragma unroll
-        for (int c = 0; c < 4; ++c)
-          tmem_ld32(col_s + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
-        tmem_wait_ld();
-        reg_fence(sr);
+      for (int c = 0; c < 4; ++c)
+        tmem_ld32(col_s + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
+      tmem_wait_ld();
+      reg_fence(sr);
+      if constexpr (!FAST) {
 #pragma unroll
         for (int c = 0; c < BN; ++c) {
           float x = __uint_as_float(sr[c]) * p.scale_log2;
           if constexpr (BIAS == kBiasDense) x = fmaf(__ldg(brow + min(kbase + c, len_k - 1)), kLog2e, x);
           if constexpr (BIAS == kBiasAlibi) x = fmaf(neg_slope2, fabsf(static_cast<float>(kbase + c - i - diag)), x);
-          if (edge && (c >= hi || c < lo)) x = -INFINITY;
           sr[c] = __float_as_uint(x);
         }
-        float mx0 = -INFINITY, mx1 = -INFINITY;
+      }
+      if (edge) {
 #pragma unroll
-        for (int c = 0; c < BN; c += 2) {
-          mx0 = fmaxf(mx0, __uint_as_float(sr[c]));
-          mx1 = fmaxf(mx1, __uint_as_float(sr[c + 1]));
-        }
-        const float mx = fmaxf(mx0, mx1);
-        const bool move = mx > m + kRescaleThreshold;
-        m_next = move ? mx : m;
-        alpha = move ? ex2(m - m_next) : 1.f;
-        const float neg_m = m_next == -INFINITY ? 0.f : -m_next;
+        for (int c = 0; c < BN; ++c)
+          if (c >= hi || c < lo) sr[c] = 0xff800000u;  // -inf
+      }
+      float mx0 = -INFINITY, mx1 = -INFINITY;
+#pragma unroll
+      for (int c = 0; c < BN; c += 2) {
+        mx0 = fmaxf(mx0, __uint_as_float(sr[c]));
+        mx1 = fmaxf(mx1, __uint_as_float(sr[c + 1]));
+      }
+      float mx = fmaxf(mx0, mx1);
+      if constexpr (FAST) mx *= sc2;  // scale > 0: max commutes with it
+      const bool move = mx > m + kRescaleThreshold;
+      m_next = move ? mx : m;
+      alpha = move ? ex2(m - m_next) : 1.f;
+      const float neg_m = m_next == -INFINITY ? 0.f : -m_next;
+      // P over the score columns already read: 32 keys -> 16 bf16 pairs per
+      // store (P chunk c covers columns [16c, 16c + 16), scores already read).
+      // EMU: on tiles with no hidden key (every score finite) one pair in
+      // kEmuEvery takes the FMA-pipe exponential instead of the MUFU one.
+      auto exps = [&](auto emu) {
+        constexpr bool EMU = decltype(emu)::value;
 #pragma unroll
         for (int c = 0; c < 4; ++c) {
           uint32_t pk[16];
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
-            const float p0 = ex2(__uint_as_float(sr[c * 32 + 2 * e]) + neg_m);
-            const float p1 = ex2(__uint_as_float(sr[c * 32 + 2 * e + 1]) + neg_m);
+            const float x0 = __uint_as_float(sr[c * 32 + 2 * e]), x1 = __uint_as_float(sr[c * 32 + 2 * e + 1]);
+            const float a0 = FAST ? fmaf(x0, sc2, neg_m) : x0 + neg_m;
+            const float a1 = FAST ? fmaf(x1, sc2, neg_m) : x1 + neg_m;
+            float p0, p1;
+            if (EMU && e % kEmuEvery == kEmuEvery - 1) {
+              p0 = ex2_poly(a0);
+              p1 = ex2_poly(a1);
+            } else {
+              p0 = ex2(a0);
+              p1 = ex2(a1);
+            }
             rs0 += p0;
             rs1 += p1;
             pk[e] = pack_bf16(p0, p1);
           }
           tmem_st16(col_s + c * 16, pk);
         }
+      };
+      if constexpr (kEmuEvery > 0) {
+        if (!edge)
+          exps(std::true_type{});
+        else
+          exps(std::false_type{});
+      } else {
+        exps(std::false_type{});
       }
       l = l * alpha + (rs0 + rs1);
       m = m_next;
@@ -502,11 +461,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D, int DV, int BIAS, bool FAST, bool PARTIAL>
+template <int D, int DV, int BIAS, bool FAST, bool PARTIAL, bool QK8 = false>
 int launch_pp_t(const TcGeom& g, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                 const FwdParams& p, cudaStream_t st) {
-  const size_t smem = sizeof(PPSmem<D, DV>) + 1024;
-  auto kern = fwd_pp_kernel<D, DV, BIAS, FAST, PARTIAL>;
+  const size_t smem = sizeof(PPSmem<D, DV, QK8>) + 1024;
+  auto kern = fwd_pp_kernel<D, DV, BIAS, FAST, PARTIAL, QK8>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return ATTN_ERR_CUDA;
   const int max_nq = g.cu_q ? g.max_nq : g.Nq;
@@ -538,6 +497,13 @@ int dispatch_pp(const TcGeom& g, const CUtensorMap& mq, const CUtensorMap& mk, c
 }
 
 }  // namespace
+
+int launch_fwd_pp_fp8(const TcGeom& g, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                      const FwdParams& p, cudaStream_t st) {
+  if (g.D != 128 || (g.Dv && g.Dv != 128) || g.cu_q || g.bias || g.alibi || !(g.scale > 0.f))
+    return ATTN_ERR_UNSUPPORTED;
+  return launch_pp_t<128, 128, kBiasNone, true, false, true>(g, mq, mk, mv, p, st);
+}
 
 int launch_fwd_pp(const TcGeom& g, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                   const FwdParams& p, int bias_kind, bool fast, bool partial, cudaStream_t st) {

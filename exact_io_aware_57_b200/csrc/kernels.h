@@ -100,6 +100,8 @@ struct FwdParams {
   float* o_part;                       // [num_splits, B, Nq, Hq, D] fp32, or null: O in bf16 to o
   float* lse_part;                     // [num_splits, B, Hq, Nq]
   long long part_o_stride, part_lse_stride;
+  const float* q_scale;  // FP8 forward: per-(batch, head) e4m3 scales of Q [B, Hq] and K [B, Hkv]
+  const float* k_scale;
   int* status;
   long long wait_limit;
 };
@@ -110,6 +112,26 @@ struct FwdParams {
 // partials to p.o_part / p.lse_part.
 int launch_fwd_pp(const TcGeom& g, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                   const FwdParams& p, int bias_kind, bool fast, bool partial, cudaStream_t st);
+// Forward with one 128-row query tile per CTA whose softmax is split over the
+// keys between two warpgroups (fwd_sk_sm100.cu); same arguments.
+int launch_fwd_sk(const TcGeom& g, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                  const FwdParams& p, int bias_kind, bool fast, bool partial, cudaStream_t st);
+int launch_fwd_sk_fp8(const TcGeom& g, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                      const FwdParams& p, cudaStream_t st);
+// The same kernel with e4m3 Q/K tiles (maps over the quantised tensors).
+int launch_fwd_pp_fp8(const TcGeom& g, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                      const FwdParams& p, cudaStream_t st);
+// FwdParams of a forward launch (everything but the tensor maps).
+int fwd_params(const TcGeom& g, __nv_bfloat16* o, float* lse, const SplitKV* split, FwdParams& p);
+
+// Per-(batch, head) e4m3 quantisation of x [B, N, H, D] (bf16): scales[b, h] =
+// amax / 448 (1 when amax = 0), x8 = e4m3(x / scale) (fp32 quotient, RNE, saturated).
+int launch_quantize_e4m3(const __nv_bfloat16* x, uint8_t* x8, float* scales, int B, int N, int H, int D,
+                         cudaStream_t st);
+// FP8 forward: S = Q8 K8^T on e4m3 tensor cores, scaled by q_scale * k_scale;
+// P V in bf16.  Dense inputs, D = DV = 128, no bias, positive scale.
+int launch_fwd_fp8(const TcGeom& g, const void* q8, const float* q_scale, const void* k8, const float* k_scale,
+                   __nv_bfloat16* o, float* lse, cudaStream_t st);
 
 int launch_fwd_sm100(const TcGeom& g, __nv_bfloat16* o, float* lse, cudaStream_t st, const SplitKV* split = nullptr);
 // O = sum_t exp(LSE_t - LSE) O_t, LSE = log sum_t exp(LSE_t) over num_parts

@@ -32,6 +32,7 @@ class Workload:
     len_hi: int = 0
     n_q: int = 0              # query length when it differs from n (the key length)
     splitkv: bool = False     # forward through the split-KV path
+    fp8: bool = False         # Q, K quantised to e4m3 per (batch, head); S on e4m3 tensor cores, P V in bf16
     description: str = field(default="", compare=False)
 
 
@@ -53,6 +54,10 @@ WORKLOADS = {
                     "bf16", True, False, n_q=512, splitkv=True,
                     description="a 512-query block at the end of a 65536-key sequence (bottom-right causal), "
                                 "GQA 32:8: 128 query-tile CTAs alone would not fill 148 SMs"),
+    "c3fp8": Workload("FP8 causal B=2 H=32 N=8192 d=128 fwd (e4m3 Q/K, bf16 P V)", 2, 32, 32, 8192, 128, "e4m3+bf16",
+                      True, False, sigma_qk=3.0, fp8=True,
+                      description="the causal workload's forward with per-head e4m3 quantisation of Q and K "
+                                  "inside the step"),
     "c5b": Workload("single sequence causal bf16 N=32768 H=16 d=128 fwd", 1, 16, 16, 32768, 128, "bf16",
                     True, False,
                     description="one sequence of 32768 tokens, 16 heads, causal, forward"),

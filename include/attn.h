@@ -132,12 +132,22 @@ int attn_bwd_local(const void* q, const void* k, const void* v, const float* ali
  * 0.2 Notation: V and O have d_v columns, Q and K have d): v is
  * [batch, n_k, h_kv, d_v] and o is [batch, n_q, h_q, d_v], d and d_v each in
  * {64, 128}.  d_v == d is attn_fwd without a bias; d_v != d takes bf16 only
- * (ATTN_ERR_UNSUPPORTED for fp32) and has no backward in this library.
- * Otherwise as attn_fwd.
+ * (ATTN_ERR_UNSUPPORTED for fp32).  Otherwise as attn_fwd.
  */
 int attn_fwd_dv(const void* q, const void* k, const void* v, void* o, float* lse, int batch,
                 int h_q, int h_kv, int n_q, int n_k, int d, int d_v, float scale, int causal,
                 int dtype, void* stream);
+
+/*
+ * Backward of attn_fwd_dv: v, o, dout, dv have width d_v, q, k, dq, dk width
+ * d.  workspace: attn_bwd_workspace_size(batch, h_q, n_q, d) bytes (the dQ
+ * accumulator has width d).  d_v == d is attn_bwd without a bias; d_v != d
+ * takes bf16 only.  Otherwise as attn_bwd.
+ */
+int attn_bwd_dv(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                const void* dout, void* dq, void* dk, void* dv, void* workspace,
+                size_t workspace_bytes, int batch, int h_q, int h_kv, int n_q, int n_k, int d,
+                int d_v, float scale, int causal, int dtype, void* stream);
 
 /*
  * Backward of attn_fwd_varlen (packed sequences, same layouts and offsets):
@@ -205,6 +215,31 @@ int attn_merge_partials(const float* o_parts, const float* lse_parts, int num_pa
 int attn_fwd_partial(const void* q, const void* k, const void* v, float* o_part, float* lse_part,
                      int batch, int h_q, int h_kv, int n_q, int n_k, int d, float scale, int causal,
                      int dtype, void* stream);
+
+/*
+ * FP8 forward ("Understanding FlashAttention Pt 1", contents 5.6: FP8 buys
+ * speed at a stated cost in precision).  Q and K are first quantised per
+ * (batch, head) by attn_quantize_e4m3; S = Q8 K8^T then runs on the e4m3
+ * tensor cores (fp32 accumulation) and is rescaled by q_scale * k_scale, while
+ * P V stays in bf16.  The result is the exact attention of the dequantised
+ * inputs Q8 * q_scale, K8 * k_scale and V, to the bf16 tolerances of attn_fwd.
+ *
+ * attn_quantize_e4m3: x bf16 [batch, n, heads, d] (d in {64, 128}) ->
+ *   scales fp32 [batch, heads], scale = amax / 448 over that (batch, head)
+ *   (fp32 division; 1 when the head is all zeros), and x8 e4m3 bytes of the
+ *   same layout, x8 = e4m3(x / scale) with the quotient in fp32 (IEEE
+ *   division), rounded to nearest even and saturated at +-448.  x8 and x
+ *   16-byte aligned.
+ * attn_fwd_fp8: q8 [batch, n_q, h_q, d], k8 [batch, n_k, h_kv, d] (e4m3 bytes),
+ *   their scales [batch, h_q] / [batch, h_kv], v bf16 [batch, n_k, h_kv, d];
+ *   o bf16 and lse as attn_fwd.  d = 128, scale > 0, no bias (otherwise
+ *   ATTN_ERR_UNSUPPORTED).
+ */
+int attn_quantize_e4m3(const void* x, void* x8, float* scales, int batch, int n, int heads, int d,
+                       void* stream);
+int attn_fwd_fp8(const void* q8, const float* q_scales, const void* k8, const float* k_scales,
+                 const void* v, void* o, float* lse, int batch, int h_q, int h_kv, int n_q, int n_k,
+                 int d, float scale, int causal, void* stream);
 
 /*
  * attn_bwd without a workspace argument, for callers that cannot allocate

@@ -87,6 +87,8 @@ class Oracle:
         L.oracle_merge_partials.argtypes = [P, P, i, i, i, P, P]
         L.oracle_quantize_e4m3.argtypes = [P, ll, d, P]
         L.oracle_quantize_e4m3.restype = None
+        L.oracle_quantize_e4m3_heads.argtypes = [P, i, i, i, i, P, P]
+        L.oracle_quantize_e4m3_heads.restype = None
         for f in (L.oracle_attn_fwd, L.oracle_attn_fwd_rows, L.oracle_attn_fwd_varlen,
                   L.oracle_attn_fwd_stream, L.oracle_attn_bwd, L.oracle_merge_partials):
             f.restype = None
@@ -192,6 +194,17 @@ class Oracle:
         out = np.empty_like(x)
         self._lib.oracle_quantize_e4m3(_ptr(x), x.size, float(scale), _ptr(out))
         return out
+
+    def quantize_e4m3_heads(self, x):
+        """Per-(batch, head) e4m3 quantisation of x [B, N, H, d]: returns the
+        dequantised values (fp64, same shape) and the fp32 scales [B, H]
+        (amax / 448), the codes decided on the fp32 quotient x / scale."""
+        x = _f64(x)
+        B, N, H, d = x.shape
+        out = np.empty_like(x)
+        scales = np.empty((B, H))
+        self._lib.oracle_quantize_e4m3_heads(_ptr(x), B, N, H, d, _ptr(out), _ptr(scales))
+        return out, scales
 
     # -------------------------------------------------------------------- merge
     def merge_partials(self, o_parts, lse_parts):

@@ -413,6 +413,34 @@ void oracle_quantize_e4m3(const double* x, long long n, double scale, double* ou
 }
 
 /*
+ * Per-head quantisation of x [B, N, H, d] for the FP8 forward: for each
+ * (batch b, head h), amax = max |x| over that head's rows, scale = amax / 448
+ * (1 when amax = 0), and each element becomes e4m3(x / scale) * scale.  The
+ * scale and the quotient are taken in fp32 (IEEE division), the precision in
+ * which the kernel decides each e4m3 code, so that both sides pick the same
+ * code; the returned values and scales are exact in fp64.
+ */
+void oracle_quantize_e4m3_heads(const double* x, int B, int N, int H, int d, double* out, double* scales) {
+  for (int b = 0; b < B; ++b)
+    for (int h = 0; h < H; ++h) {
+      double amax = 0.0;
+      for (int n = 0; n < N; ++n) {
+        const double* row = x + (((long long)b * N + n) * H + h) * d;
+        for (int c = 0; c < d; ++c) if (fabs(row[c]) > amax) amax = fabs(row[c]);
+      }
+      const float scale = amax > 0.0 ? (float)amax / 448.0f : 1.0f;
+      scales[b * H + h] = scale;
+      for (int n = 0; n < N; ++n) {
+        const long long o = (((long long)b * N + n) * H + h) * d;
+        for (int c = 0; c < d; ++c) {
+          const float qf = (float)x[o + c] / scale;
+          out[o + c] = round_e4m3((double)qf) * (double)scale;
+        }
+      }
+    }
+}
+
+/*
  * Merge of partial results over disjoint key shards: shard t holds the exact
  * attention (o_t, lse_t) of the row over its own keys only.  The combined row
  * follows from the same rescale-and-add recurrence as the streaming forward:

@@ -66,3 +66,26 @@ def test_attention_of_quantised_inputs_is_the_oracle_on_them(orc):
     p = np.exp(s_ - s_.max(-1, keepdims=True))
     p /= p.sum(-1, keepdims=True)
     assert np.allclose(o, np.einsum("bhij,bjhc->bihc", p, v), atol=1e-13)
+
+
+def test_per_head_quantiser_against_numpy_and_torch(orc):
+    """oracle_quantize_e4m3_heads: the scale of each (batch, head) is fp32 amax / 448
+    (numpy's fp32 division), and every code is torch's fp32 -> e4m3 cast of the
+    fp32 quotient (clamped to the finite range first: the oracle saturates)."""
+    rng = np.random.default_rng(5)
+    x = torch.from_numpy(rng.standard_normal((2, 37, 3, 64)) * 4.0).to(torch.bfloat16)
+    x[1, :, 2] = 0                                     # an all-zero head: scale 1, codes 0
+    x[0, 5, 1, 7] = 300.0                              # one large entry sets its head's scale
+    got, scales = orc.quantize_e4m3_heads(x)
+    xf = x.float()
+    amax = xf.abs().amax(dim=(1, 3))                   # [B, H], exact
+    a32 = amax.numpy().astype(np.float32)
+    sc = torch.from_numpy(np.where(a32 > 0, a32 / np.float32(448.0), np.float32(1.0)).astype(np.float32))
+    assert np.array_equal(scales, sc.double().numpy())
+    quot = xf / sc[:, None, :, None]                   # fp32 IEEE division, as the kernel
+    ref = quot.clamp(-448, 448).to(torch.float8_e4m3fn).double() * sc[:, None, :, None].double()
+    assert np.array_equal(got, ref.numpy())
+    assert not got[1, :, 2].any() and scales[1, 2] == 1.0
+    # the largest magnitude of every head maps onto 448 * scale (up to the fp32 rounding of the scale)
+    top = np.abs(got).max(axis=(1, 3))
+    assert np.all(np.abs(top - amax.double().numpy()) <= 2.0 ** -4 * amax.double().numpy() + 1e-30)

@@ -63,7 +63,7 @@ def _worker(rank, world, port, causal, out):
 @pytest.mark.parametrize("world", [2, 3])
 @pytest.mark.parametrize("causal", [False, True])
 def test_ring_forward_equals_one_shot(world, causal):
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()
     out = mgr.dict()
     mp.spawn(_worker, args=(world, _free_port(), causal, out), nprocs=world, join=True)
     for r in range(world):
