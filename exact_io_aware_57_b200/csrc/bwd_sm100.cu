@@ -22,21 +22,22 @@
 //               takes queries [64g, 64g+64) of P^T / dS^T and columns
 //               [gD/2, (g+1)D/2) of dQ, dK and dV, so every SM sub-partition
 //               runs two warps of each elementwise phase.
-// TMEM columns: [0,128) S^T (then P^T as bf16 pairs in [0,64)),
-//   [128,256) dP^T (then the dQ tile), [256,256+D) dV, [256+D,256+2D) dK.
+// D is the width of Q, K, dQ, dK and DV that of V, O, dO, dV (equal except
+// for attn_bwd_dv).  TMEM columns: [0,128) S^T (then P^T as bf16 pairs in
+// [0,64)), [128,256) dP^T (then the dQ tile), [256,256+DV) dV,
+// [256+DV,256+DV+D) dK.
 // Per step (query head h, query tile i):
-//   MMA   S^T = K_j Q_i^T and dP^T = V_j dO_i^T, interleaved (once the previous
-//         dQ has left TMEM)
-//   WGs   P^T = 2^(scale log2e S^T + log2e B^T - log2e LSE) -> TMEM (bf16);
+//   MMA   S^T = K_j Q_i^T, committed alone; then dP^T = V_j dO_i^T once the
+//         previous dQ has left TMEM
+//   WGs   P^T = 2^(scale log2e S^T + log2e B^T - log2e LSE) -> TMEM (bf16),
+//         overlapping the dP^T MMAs;
 //         dS^T = P^T o (dP^T - D) -> shared memory (bf16, 128B-swizzled)
 //   MMA   dV += P^T dO_i (P^T from TMEM), dK += dS^T Q_i and dQ_i = dS K_j,
-//         interleaved
+//         round-robin over the three accumulators
 //   WGs   dQ_i -> the step's own Q_i/dO_i buffers (free once its MMAs are done);
 //         the producer adds them into the fp32 accumulator with TMA bulk
 //         reductions and refills the buffers only after those have read them,
 //         so the reduction overlaps the next step instead of holding it up.
-// A chain of MMAs into one TMEM accumulator waits on each previous result;
-// every group above interleaves two or three accumulators instead.
 #include <algorithm>
 
 #include "common.cuh"
@@ -52,15 +53,13 @@ constexpr int NSTQ = 2;   // Q/dO stages
 constexpr int kThreads = 320;
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kColST = 0, kColDPT = 128, kColDV = 256;
+// One exponential of P^T in kBwdEmuEvery goes to the FMA pipe (ex2_poly) on
+// tiles without a mask (measured: 1 in 8 helps a little, 1 in 4 hurts).
 #ifndef ATTN_BWD_EX2_EMU_EVERY
-#define ATTN_BWD_EX2_EMU_EVERY 0
+#define ATTN_BWD_EX2_EMU_EVERY 8
 #endif
 constexpr int kBwdEmuEvery = ATTN_BWD_EX2_EMU_EVERY;
-#ifndef ATTN_BWD_SPLIT_SDP
-#define ATTN_BWD_SPLIT_SDP 0
-#endif
-// Issue S^T and dP^T one after the other (committed apart) instead of interleaved.
-constexpr bool kSplitSdp = ATTN_BWD_SPLIT_SDP != 0;
+
 
 // D: width of Q, K, dQ, dK; DV: width of V, O, dO, dV.  The fp32 dQ tile of a
 // step (D / 32 boxes of 128 rows x 32 columns, 16 KB each) is staged in that
@@ -412,50 +411,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t q_addr = smem_u32(s.q[st]), do_addr = smem_u32(s.dout[st]);
         // S^T = K_j Q_i^T (over P^T of the previous step, whose dV MMA was issued
-        // earlier by this thread: tcgen05.mma executes in issue order) and
-        // dP^T = V_j dO_i^T, round-robin.  dP^T goes where dQ of the previous
-        // step was: the first S^T MMA is issued before waiting for it to leave.
-        if constexpr (kSplitSdp) {
-          // S^T alone first (the elementwise groups start P^T on it), then
-          // dP^T once the previous dQ has left TMEM
+        // earlier by this thread: tcgen05.mma executes in issue order), committed
+        // on its own so that the elementwise groups start P^T on it; then
+        // dP^T = V_j dO_i^T, where dQ of the previous step was, once that has
+        // left TMEM.  Issuing the two apart costs nothing on the tensor pipe and
+        // lets the exponentials of P^T overlap dP^T.
 #pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
-            mma_ss(tmem + kColST, sdesc_sw128(k_addr + off, 16, 1024), sdesc_sw128(q_addr + off, 16, 1024), idesc_s,
-                   kk > 0);
-          }
-          // its completion also implies that the previous step's MMAs, the last
-          // readers of the dS^T tile, are done
-          mma_commit(&s.st_full);
-          if (step > 0 && !mbar_wait(&s.tmem_free, (step - 1) & 1, ab)) break;
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < DV / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
-            mma_ss(tmem + kColDPT, sdesc_sw128(v_addr + off, 16, 1024), sdesc_sw128(do_addr + off, 16, 1024),
-                   idesc_s, kk > 0);
-          }
-          mma_commit(&s.dp_full);
-        } else {
-          mma_ss(tmem + kColST, sdesc_sw128(k_addr, 16, 1024), sdesc_sw128(q_addr, 16, 1024), idesc_s, false);
-          if (step > 0 && !mbar_wait(&s.tmem_free, (step - 1) & 1, ab)) break;
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < (D > DV ? D : DV) / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
-            const uint32_t off1 = ((kk + 1) >> 2) * (128 * 128) + ((kk + 1) & 3) * 32;
-            if (kk < DV / 16)
-              mma_ss(tmem + kColDPT, sdesc_sw128(v_addr + off, 16, 1024), sdesc_sw128(do_addr + off, 16, 1024),
-                     idesc_s, kk > 0);
-            if (kk + 1 < D / 16)
-              mma_ss(tmem + kColST, sdesc_sw128(k_addr + off1, 16, 1024), sdesc_sw128(q_addr + off1, 16, 1024),
-                     idesc_s, true);
-          }
-          // its completion also implies that the previous step's MMAs, the last
-          // readers of the dS^T tile, are done
-          mma_commit(&s.st_full);
-          mma_commit(&s.dp_full);
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+          mma_ss(tmem + kColST, sdesc_sw128(k_addr + off, 16, 1024), sdesc_sw128(q_addr + off, 16, 1024), idesc_s,
+                 kk > 0);
         }
+        // its completion also implies that the previous step's MMAs, the last
+        // readers of the dS^T tile, are done
+        mma_commit(&s.st_full);
+        if (step > 0 && !mbar_wait(&s.tmem_free, (step - 1) & 1, ab)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < DV / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
+          mma_ss(tmem + kColDPT, sdesc_sw128(v_addr + off, 16, 1024), sdesc_sw128(do_addr + off, 16, 1024), idesc_s,
+                 kk > 0);
+        }
+        mma_commit(&s.dp_full);
         if (!mbar_wait(&s.ds_ready, step & 1, ab)) break;
         tc_fence_after();
         // dV += P^T dO_i (P^T from TMEM), dK += dS^T Q_i and dQ_i = dS K_j (the

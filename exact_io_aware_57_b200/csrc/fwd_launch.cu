@@ -72,13 +72,8 @@ int launch_fwd_sm100(const TcGeom& g, __nv_bfloat16* o, float* lse, cudaStream_t
   // FAST: no bias and a positive scale, so the row max can be taken on raw scores
   const bool fast = !g.bias && !g.alibi && g.scale > 0.f;
   if (dv != g.D && (split || g.bias || g.alibi)) return ATTN_ERR_UNSUPPORTED;
-#ifdef ATTN_FWD_PINGPONG
   return launch_fwd_pp(g, mq, mk, mv, p, g.bias ? kBiasDense : g.alibi ? kBiasAlibi : kBiasNone, fast,
                        split != nullptr, st);
-#else
-  return launch_fwd_sk(g, mq, mk, mv, p, g.bias ? kBiasDense : g.alibi ? kBiasAlibi : kBiasNone, fast,
-                       split != nullptr, st);
-#endif
 }
 
 }  // namespace attn
@@ -106,11 +101,7 @@ int launch_fwd_fp8(const TcGeom& g, const void* q8, const float* q_scale, const 
   if (fwd_params(g, o, lse, nullptr, p) != ATTN_OK) return ATTN_ERR_CUDA;
   p.q_scale = q_scale;
   p.k_scale = k_scale;
-#ifdef ATTN_FWD_PINGPONG
   return launch_fwd_pp_fp8(g, mq, mk, mv, p, st);
-#else
-  return launch_fwd_sk_fp8(g, mq, mk, mv, p, st);
-#endif
 }
 
 }  // namespace attn

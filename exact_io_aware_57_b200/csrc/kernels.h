@@ -112,12 +112,6 @@ struct FwdParams {
 // partials to p.o_part / p.lse_part.
 int launch_fwd_pp(const TcGeom& g, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                   const FwdParams& p, int bias_kind, bool fast, bool partial, cudaStream_t st);
-// Forward with one 128-row query tile per CTA whose softmax is split over the
-// keys between two warpgroups (fwd_sk_sm100.cu); same arguments.
-int launch_fwd_sk(const TcGeom& g, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                  const FwdParams& p, int bias_kind, bool fast, bool partial, cudaStream_t st);
-int launch_fwd_sk_fp8(const TcGeom& g, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                      const FwdParams& p, cudaStream_t st);
 // The same kernel with e4m3 Q/K tiles (maps over the quantised tensors).
 int launch_fwd_pp_fp8(const TcGeom& g, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                       const FwdParams& p, cudaStream_t st);
