@@ -252,6 +252,17 @@ ATTN_DEVINL uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
          (static_cast<uint64_t>((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
 }
 
+// Per-warpgroup register budgets (every warp of the warpgroup executes the same
+// one): dec hands registers back to the CTA's pool, inc waits for them.
+template <uint32_t N>
+ATTN_DEVINL void setmaxnreg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <uint32_t N>
+ATTN_DEVINL void setmaxnreg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+
 // ---------------------------------------------------------------------- math
 ATTN_DEVINL float ex2(float x) {
   float y;

@@ -41,7 +41,6 @@
 // Split-KV: with num_splits > 1 the grid's z index also runs over key ranges;
 // each CTA then writes O_t (normalised, fp32) and LSE_t for the merge.
 #include <algorithm>
-#include <type_traits>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -52,7 +51,20 @@ namespace {
 
 constexpr int BM = 128;  // query rows per tile (two tiles per CTA)
 constexpr int BN = 128;  // keys per KV tile
-constexpr int kThreads = 320;
+#ifndef ATTN_FWD_REG_SPLIT
+#define ATTN_FWD_REG_SPLIT 0
+#endif
+// Register split: 12 warps launched at 168 registers a thread (384 x 168 =
+// 64,512 of the 65,536); warps 8..11 (MMA, TMA, two idle) give theirs down to
+// 88 and the two softmax warpgroups take 208: 4 x 32 x 88 + 8 x 32 x 208 =
+// 64,512, the launch's pool, and per SM sub-partition (three warps) 2 x 32 x
+// 208 + 32 x 88 = 16,128 of its 16,384.  Without it: 10 warps, 168 registers.
+constexpr bool kRegSplit = ATTN_FWD_REG_SPLIT != 0;
+constexpr int kThreads = kRegSplit ? 384 : 320;
+constexpr int kLaunchRegs = 168, kLowRegs = 88, kHighRegs = 208;
+static_assert(!kRegSplit || (4 * 32 * kLowRegs + 8 * 32 * kHighRegs == kThreads * kLaunchRegs &&
+                             2 * 32 * kHighRegs + 32 * kLowRegs <= 16384),
+              "register split must match the launch's pool");
 constexpr int kWarpMma = 8, kWarpLoad = 9;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.f;  // log2 units: P stays <= 256
@@ -178,6 +190,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const Abort ab{&s.abort_flag, p.status, p.wait_limit};
 
   if (warp == kWarpLoad) {
+    if constexpr (kRegSplit) setmaxnreg_dec<kLowRegs>();
     // ===================================================== TMA producer
     if (lane == 0 && n_union > 0) {
       tma_prefetch_desc(&tm_q);
@@ -219,6 +232,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp == kWarpMma) {
+    if constexpr (kRegSplit) setmaxnreg_dec<kLowRegs>();
     // ===================================================== MMA issuer
     if (lane == 0 && n_union > 0) {
       constexpr uint32_t idesc_s = idesc_bf16(BM, BN, 0, 0);   // Q_t: K-major, K_j: K-major
@@ -276,7 +290,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mma_commit(&s.drain);
       mbar_wait_drain(&s.drain, 0, p.wait_limit);
     }
-  } else {
+  } else if (warp < 8) {
+    if constexpr (kRegSplit) setmaxnreg_inc<kHighRegs>();
     // ===================================================== softmax warpgroups
     const int t = warp >> 2;       // query tile of this warpgroup
     const int quarter = warp & 3;  // TMEM lanes [32 quarter, 32 quarter + 32)
@@ -346,38 +361,31 @@ __global__ void __launch_bounds__(kThreads, 1)
       // store (P chunk c covers columns [16c, 16c + 16), scores already read).
       // EMU: on tiles with no hidden key (every score finite) one pair in
       // kEmuEvery takes the FMA-pipe exponential instead of the MUFU one.
-      auto exps = [&](auto emu) {
-        constexpr bool EMU = decltype(emu)::value;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t pk[16];
+      for (int c = 0; c < 4; ++c) {
+        uint32_t pk[16];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const float x0 = __uint_as_float(sr[c * 32 + 2 * e]), x1 = __uint_as_float(sr[c * 32 + 2 * e + 1]);
-            const float a0 = FAST ? fmaf(x0, sc2, neg_m) : x0 + neg_m;
-            const float a1 = FAST ? fmaf(x1, sc2, neg_m) : x1 + neg_m;
-            float p0, p1;
-            if (EMU && e % kEmuEvery == kEmuEvery - 1) {
-              p0 = ex2_poly(a0);
-              p1 = ex2_poly(a1);
-            } else {
-              p0 = ex2(a0);
-              p1 = ex2(a1);
-            }
-            rs0 += p0;
-            rs1 += p1;
-            pk[e] = pack_bf16(p0, p1);
+        for (int e = 0; e < 16; ++e) {
+          const float x0 = __uint_as_float(sr[c * 32 + 2 * e]), x1 = __uint_as_float(sr[c * 32 + 2 * e + 1]);
+          const float a0 = FAST ? fmaf(x0, sc2, neg_m) : x0 + neg_m;
+          const float a1 = FAST ? fmaf(x1, sc2, neg_m) : x1 + neg_m;
+          float p0, p1;
+          // FAST: one pair in kEmuEvery on the FMA pipe.  A hidden key (-inf)
+          // then gives about 2^-126 instead of 0: harmless next to a row's
+          // largest p (>= 2^-8 under the reference-max rule), and a row with no
+          // visible key at all is recognised in the epilogue by m = -inf
+          if (FAST && kEmuEvery > 0 && e % (kEmuEvery > 0 ? kEmuEvery : 1) == kEmuEvery - 1) {
+            p0 = ex2_poly(a0);
+            p1 = ex2_poly(a1);
+          } else {
+            p0 = ex2(a0);
+            p1 = ex2(a1);
           }
-          tmem_st16(col_s + c * 16, pk);
+          rs0 += p0;
+          rs1 += p1;
+          pk[e] = pack_bf16(p0, p1);
         }
-      };
-      if constexpr (kEmuEvery > 0) {
-        if (!edge)
-          exps(std::true_type{});
-        else
-          exps(std::false_type{});
-      } else {
-        exps(std::false_type{});
+        tmem_st16(col_s + c * 16, pk);
       }
       l = l * alpha + (rs0 + rs1);
       m = m_next;
@@ -404,7 +412,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (ok && my.n > 0) ok = __all_sync(0xffffffffu, mbar_wait(&s.o_done[t], 0, ab));
     tc_fence_after();
     if (ok) {
-      const float inv_l = l > 0.f ? 1.f / l : 0.f;
+      // a row with no visible key (m never left -inf) is empty
+      const bool empty = !(l > 0.f) || m == -INFINITY;
+      const float inv_l = empty ? 0.f : 1.f / l;
       __nv_bfloat16* orow = p.o + bidx * p.o_bstride + ((long long)(q_off + i) * p.Hq + h) * DV;
       float* prow = nullptr;
       if constexpr (PARTIAL)
@@ -442,13 +452,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       if (row_ok) {
-        const float lse = l > 0.f ? (m + __log2f(l)) * kLn2 : -INFINITY;
+        const float lse = empty ? -INFINITY : (m + __log2f(l)) * kLn2;
         if constexpr (PARTIAL)
           p.lse_part[split * p.part_lse_stride + bidx * p.lse_bstride + (long long)h * p.lse_hstride + q_off + i] = lse;
         else
           p.lse[bidx * p.lse_bstride + (long long)h * p.lse_hstride + q_off + i] = lse;
       }
     }
+  } else {
+    if constexpr (kRegSplit) setmaxnreg_dec<kLowRegs>();  // warps 10, 11: idle
   }
 
   // ---- teardown
@@ -466,6 +478,12 @@ int launch_pp_t(const TcGeom& g, const CUtensorMap& mq, const CUtensorMap& mk, c
                 const FwdParams& p, cudaStream_t st) {
   const size_t smem = sizeof(PPSmem<D, DV, QK8>) + 1024;
   auto kern = fwd_pp_kernel<D, DV, BIAS, FAST, PARTIAL, QK8>;
+  if constexpr (kRegSplit) {
+    // the split adds up only against a launch of exactly kLaunchRegs a thread
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, kern) != cudaSuccess) return ATTN_ERR_CUDA;
+    if (fa.numRegs != kLaunchRegs) return ATTN_ERR_UNSUPPORTED;
+  }
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return ATTN_ERR_CUDA;
   const int max_nq = g.cu_q ? g.max_nq : g.Nq;
