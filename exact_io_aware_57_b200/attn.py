@@ -44,6 +44,7 @@ EXPORTS = {
     "attn_bwd_dv": (_I, [_VP, _VP, _VP, _VP, _FP, _VP, _VP, _VP, _VP, _VP, _SZ, _I, _I, _I, _I, _I, _I, _I, _F,
                          _I, _I, _VP]),
     "attn_selftest_wait_timeout": (_I, [ctypes.c_longlong, _VP]),
+    "attn_selftest_ex2": (_I, [_VP, _VP, ctypes.c_longlong, _VP]),
     "attn_splitkv_num_splits": (_I, [_I, _I, _I, _I]),
     "attn_splitkv_workspace_size": (_SZ, [_I, _I, _I, _I, _I]),
     "attn_fwd_splitkv": (_I, [_VP, _VP, _VP, _VP, _FP, _I, _I, _I, _I, _I, _I, _F, _I, _I, _VP, _SZ, _I, _VP]),
@@ -209,6 +210,15 @@ def attn_bwd_dv(q, k, v, o, lse, dout, causal=False, scale=None, workspace=None,
 def attn_selftest_wait_timeout(limit_cycles=1_000_000, stream=None) -> None:
     """Launch the bounded-wait self-test (a wait that gives up after limit_cycles)."""
     _check(_lib.attn_selftest_wait_timeout(int(limit_cycles), _stream(stream)))
+
+
+def attn_selftest_ex2(x, stream=None):
+    """2^x by the kernels' FMA-pipe exponential (fp32 device tensor in, same out)."""
+    if x.dtype != torch.float32 or not x.is_contiguous():
+        raise ValueError("x must be a contiguous fp32 tensor")
+    y = torch.empty_like(x)
+    _check(_lib.attn_selftest_ex2(_dev(x, "x"), _dev(y, "y"), x.numel(), _stream(stream)))
+    return y
 
 
 def attn_splitkv_num_splits(batch, h_q, n_q, n_k) -> int:

@@ -619,6 +619,13 @@ int attn_selftest_wait_timeout(long long limit_cycles, void* stream) {
   return launch_wait_selftest(limit_cycles, static_cast<cudaStream_t>(stream));
 }
 
+int attn_selftest_ex2(const float* x, float* y, long long n, void* stream) {
+  if (n < 0 || (n > 0 && (!x || !y))) return ATTN_ERR_INVALID;
+  if (n == 0) return ATTN_OK;
+  if (!supported_device()) return ATTN_ERR_UNSUPPORTED;
+  return launch_ex2_selftest(x, y, n, static_cast<cudaStream_t>(stream));
+}
+
 int attn_set_kernel_events(int which, void* start, void* stop) {
   if (which != ATTN_KERNEL_FWD && which != ATTN_KERNEL_BWD) return ATTN_ERR_INVALID;
   if ((start == nullptr) != (stop == nullptr)) return ATTN_ERR_INVALID;

@@ -27,13 +27,16 @@
 // [0,64)), [128,256) dP^T (then the dQ tile), [256,256+DV) dV,
 // [256+DV,256+DV+D) dK.
 // Per step (query head h, query tile i):
-//   MMA   S^T = K_j Q_i^T, committed alone; then dP^T = V_j dO_i^T once the
-//         previous dQ has left TMEM
+//   MMA   dP^T = V_j dO_i^T once the previous dQ has left TMEM (S^T of this step
+//         was issued earlier, see below)
 //   WGs   P^T = 2^(scale log2e S^T + log2e B^T - log2e LSE) -> TMEM (bf16),
-//         overlapping the dP^T MMAs;
+//         overlapping the dP^T MMAs; P^T also stays in registers for dS^T;
 //         dS^T = P^T o (dP^T - D) -> shared memory (bf16, 128B-swizzled)
-//   MMA   dV += P^T dO_i (P^T from TMEM), dK += dS^T Q_i and dQ_i = dS K_j,
-//         round-robin over the three accumulators
+//   MMA   dV += P^T dO_i (P^T from TMEM) once P^T is there, overlapping dS^T;
+//         S^T of the next step = K_j Q_{i+1}^T as soon as Q_{i+1} has arrived
+//         (the scores columns are free once P^T has been read out), so the
+//         elementwise groups find the next scores ready; then dK += dS^T Q_i
+//         and dQ_i = dS K_j, round-robin
 //   WGs   dQ_i -> the step's own Q_i/dO_i buffers (free once its MMAs are done);
 //         the producer adds them into the fp32 accumulator with TMA bulk
 //         reductions and refills the buffers only after those have read them,
@@ -59,12 +62,6 @@ constexpr uint32_t kColST = 0, kColDPT = 128, kColDV = 256;
 #define ATTN_BWD_EX2_EMU_EVERY 8
 #endif
 constexpr int kBwdEmuEvery = ATTN_BWD_EX2_EMU_EVERY;
-#ifndef ATTN_BWD_DV_EARLY
-#define ATTN_BWD_DV_EARLY 0
-#endif
-// Issue dV += P^T dO before dS^T is ready (it only needs P^T).
-constexpr bool kDvEarly = ATTN_BWD_DV_EARLY != 0;
-
 
 // D: width of Q, K, dQ, dK; DV: width of V, O, dO, dV.  The fp32 dQ tile of a
 // step (D / 32 boxes of 128 rows x 32 columns, 16 KB each) is staged in that
@@ -143,7 +140,7 @@ ATTN_DEVINL void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
 template <bool MASK, int BIAS>
 ATTN_DEVINL void p_chunk(int c, const uint32_t (&sr)[32], uint32_t st_col, const float* nlse2, float scale_log2,
                          const float* bcol, float neg_slope2, int nk, int i0, int len_q, int kj, int len_k,
-                         int lo_off, int hi_off, int bias_diag) {
+                         int lo_off, int hi_off, int bias_diag, uint32_t (&pk)[16]) {
   const float4* nl4 = reinterpret_cast<const float4*>(nlse2 + c * 32);
   const int q0 = i0 + c * 32;
   int vis_lo = 0, vis_hi = 32;  // queries q0 + e, vis_lo <= e < vis_hi, see this key
@@ -152,7 +149,6 @@ ATTN_DEVINL void p_chunk(int c, const uint32_t (&sr)[32], uint32_t st_col, const
     vis_hi = min(min(32, len_q - q0), kj + hi_off - q0 + 1);
     if (kj >= len_k) vis_hi = 0;
   }
-  uint32_t pk[16];
 #pragma unroll
   for (int e4 = 0; e4 < 8; ++e4) {
     const float4 nl = nl4[e4];
@@ -179,10 +175,12 @@ ATTN_DEVINL void p_chunk(int c, const uint32_t (&sr)[32], uint32_t st_col, const
 // P^T of group 1 lands on S^T columns [32, 64), which group 0 reads: group 0's
 // warps arrive on `s_read` once their loads are complete and group 1 waits for
 // that phase (bounded) before it stores.  Returns false if that wait gave up.
+// keep: this thread's P^T as bf16 pairs (chunk 2g in [0,16), chunk 2g+1 in [16,32)).
 template <bool MASK, int BIAS>
 ATTN_DEVINL bool bwd_p_half(int grp, uint64_t* s_read, uint32_t parity, const Abort& ab, uint32_t st_col,
                             const float* nlse2, float scale_log2, const float* bcol, float neg_slope2, int nk, int i0,
-                            int len_q, int kj, int len_k, int lo_off, int hi_off, int bias_diag) {
+                            int len_q, int kj, int len_k, int lo_off, int hi_off, int bias_diag,
+                            uint32_t (&keep)[32]) {
   const int c0 = 2 * grp;
   uint32_t ra[32], rb[32];
   tmem_ld32(st_col + c0 * 32, ra);
@@ -199,13 +197,13 @@ ATTN_DEVINL bool bwd_p_half(int grp, uint64_t* s_read, uint32_t parity, const Ab
     tc_fence_after();
   }
   p_chunk<MASK, BIAS>(c0, ra, st_col, nlse2, scale_log2, bcol, neg_slope2, nk, i0, len_q, kj, len_k, lo_off, hi_off,
-                      bias_diag);
+                      bias_diag, *reinterpret_cast<uint32_t(*)[16]>(&keep[0]));
   p_chunk<MASK, BIAS>(c0 + 1, rb, st_col, nlse2, scale_log2, bcol, neg_slope2, nk, i0, len_q, kj, len_k, lo_off,
-                      hi_off, bias_diag);
+                      hi_off, bias_diag, *reinterpret_cast<uint32_t(*)[16]>(&keep[16]));
   return true;
 }
 
-// Phase B -- dS^T = P^T (dP^T - D) from the bf16 P^T in TMEM and dP^T, into the
+// Phase B -- dS^T = P^T (dP^T - D) from the bf16 P^T and dP^T, into the
 // 128B-swizzled shared tile (K-major for dK += dS^T Q, MN-major for dQ = dS K).
 ATTN_DEVINL void ds_chunk(int c, const uint32_t (&pr)[16], const uint32_t (&dpr)[32], const float* drow,
                           uint32_t ds_row, int r) {
@@ -235,21 +233,20 @@ ATTN_DEVINL void ds_chunk(int c, const uint32_t (&pr)[16], const uint32_t (&dpr)
   }
 }
 
-// Group g's half of phase B (its own P^T columns, chunks 2g and 2g+1).
-ATTN_DEVINL void bwd_ds_half(int grp, uint32_t st_col, uint32_t dp_col, const float* drow, uint32_t ds_row, int r) {
+// Group g's half of phase B (chunks 2g and 2g+1): dP^T from TMEM, P^T from the
+// values this thread kept in registers in phase A (`keep`), so the S^T
+// columns may already hold the next step's scores.
+ATTN_DEVINL void bwd_ds_half_kept(int grp, const uint32_t (&keep)[32], uint32_t dp_col, const float* drow,
+                                  uint32_t ds_row, int r) {
   const int c0 = 2 * grp;
-  uint32_t pa[16], da[32], pb[16], db[32];
-  tmem_ld16(st_col + c0 * 16, pa);
+  uint32_t da[32], db[32];
   tmem_ld32(dp_col + c0 * 32, da);
-  tmem_ld16(st_col + (c0 + 1) * 16, pb);
   tmem_ld32(dp_col + (c0 + 1) * 32, db);
   tmem_wait_ld();
-  reg_fence(pa);
   reg_fence(da);
-  reg_fence(pb);
   reg_fence(db);
-  ds_chunk(c0, pa, da, drow, ds_row, r);
-  ds_chunk(c0 + 1, pb, db, drow, ds_row, r);
+  ds_chunk(c0, *reinterpret_cast<const uint32_t(*)[16]>(&keep[0]), da, drow, ds_row, r);
+  ds_chunk(c0 + 1, *reinterpret_cast<const uint32_t(*)[16]>(&keep[16]), db, drow, ds_row, r);
 }
 
 template <int D, int DV, int BIAS>
@@ -414,28 +411,43 @@ __global__ void __launch_bounds__(kThreads, 1)
       constexpr uint32_t idesc_kv = idesc_bf16(BN, D, 0, 1);    // dS^T (K-major) x Q_i (MN-major)
       constexpr uint32_t idesc_dq = idesc_bf16(BM, D, 1, 1);    // dS (MN-major) x K_j (MN-major)
       const uint32_t k_addr = smem_u32(s.k), v_addr = smem_u32(s.v), ds_addr = smem_u32(s.ds);
-      bool ok = mbar_wait(&s.kv_full, 0, ab);
-      for (int step = 0; ok && step < n_steps; ++step) {
-        const int st = step % NSTQ;
-        if (!mbar_wait(&s.q_full[st], (step / NSTQ) & 1, ab)) break;
-        tc_fence_after();
-        const uint32_t q_addr = smem_u32(s.q[st]), do_addr = smem_u32(s.dout[st]);
-        // S^T = K_j Q_i^T (over P^T of the previous step, whose dV MMA was issued
-        // earlier by this thread: tcgen05.mma executes in issue order), committed
-        // on its own so that the elementwise groups start P^T on it; then
-        // dP^T = V_j dO_i^T, where dQ of the previous step was, once that has
-        // left TMEM.  Issuing the two apart costs nothing on the tensor pipe and
-        // lets the exponentials of P^T overlap dP^T.
+      // S^T(t) = K_j Q_t^T into [0, 128) (over P^T of the step before, whose dV
+      // MMA was issued earlier by this thread: tcgen05.mma executes in issue order)
+      auto s_mmas = [&](uint32_t q_addr) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
           mma_ss(tmem + kColST, sdesc_sw128(k_addr + off, 16, 1024), sdesc_sw128(q_addr + off, 16, 1024), idesc_s,
                  kk > 0);
         }
-        // its completion also implies that the previous step's MMAs, the last
-        // readers of the dS^T tile, are done
+      };
+      // The next step's scores: S^T(t + 1) over P^T(t) once dV(t) (issued before,
+      // executed in issue order) has read it; the elementwise groups keep P^T in
+      // registers for dS^T, so the S^T columns are free after the P^T phase.
+      int s_issued = 0;
+      auto next_s = [&](int t, bool block) -> bool {  // issue S^T(t) if its Q has arrived (or wait for it)
+        if (t >= n_steps || s_issued != t) return true;
+        const int st1 = t % NSTQ;
+        const uint32_t par = (t / NSTQ) & 1;
+        if (block) {
+          if (!mbar_wait(&s.q_full[st1], par, ab)) return false;
+        } else if (!mbar_try_wait(&s.q_full[st1], par)) {
+          return true;
+        }
+        tc_fence_after();
+        s_mmas(smem_u32(s.q[st1]));
+        // its completion also implies that the MMAs issued before it are done
         mma_commit(&s.st_full);
-        if (step > 0 && !mbar_wait(&s.tmem_free, (step - 1) & 1, ab)) break;
+        ++s_issued;
+        return true;
+      };
+      bool ok = mbar_wait(&s.kv_full, 0, ab);
+      if (ok) ok = next_s(0, true);
+      for (int step = 0; ok && step < n_steps; ++step) {
+        const int st = step % NSTQ;
+        const uint32_t q_addr = smem_u32(s.q[st]), do_addr = smem_u32(s.dout[st]);
+        // dP^T = V_j dO_i^T where dQ of the previous step was, once that has left
+        if (step > 0 && !(ok = mbar_wait(&s.tmem_free, (step - 1) & 1, ab))) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < DV / 16; ++kk) {
@@ -444,32 +456,31 @@ __global__ void __launch_bounds__(kThreads, 1)
                  kk > 0);
         }
         mma_commit(&s.dp_full);
-        if constexpr (kDvEarly) {
-          // dV += P^T dO_i as soon as P^T is in TMEM: it overlaps the dS^T phase
-          if (!mbar_wait(&s.pt_ready, step & 1, ab)) break;
-          tc_fence_after();
-#pragma unroll
-          for (int kk = 0; kk < BM / 16; ++kk)
-            mma_ts(tmem + kColDV, tmem + kColST + kk * 8, sdesc_sw128(do_addr + kk * 2048, BM * 128, 1024), idesc_dv,
-                   (step > 0 || kk > 0));
-        }
-        if (!mbar_wait(&s.ds_ready, step & 1, ab)) break;
+        // dV += P^T dO_i as soon as P^T is in TMEM; it overlaps the dS^T phase
+        if (!(ok = mbar_wait(&s.pt_ready, step & 1, ab))) break;
         tc_fence_after();
-        // dV += P^T dO_i (P^T from TMEM) unless issued already, dK += dS^T Q_i and
-        // dQ_i = dS K_j (the dS^T tile read MN-major), round-robin
+#pragma unroll
+        for (int kk = 0; kk < BM / 16; ++kk)
+          mma_ts(tmem + kColDV, tmem + kColST + kk * 8, sdesc_sw128(do_addr + kk * 2048, BM * 128, 1024), idesc_dv,
+                 (step > 0 || kk > 0));
+        if (!(ok = next_s(step + 1, false))) break;
+        // dK += dS^T Q_i and dQ_i = dS K_j (the dS^T tile read MN-major) once
+        // dS^T is in shared memory, round-robin
+        if (!(ok = mbar_wait(&s.ds_ready, step & 1, ab))) break;
+        if (!(ok = next_s(step + 1, false))) break;
+        tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk) {
           const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
-          if constexpr (!kDvEarly)
-            mma_ts(tmem + kColDV, tmem + kColST + kk * 8, sdesc_sw128(do_addr + kk * 2048, BM * 128, 1024), idesc_dv,
-                   (step > 0 || kk > 0));
           mma_ss(tmem + kColDK, sdesc_sw128(ds_addr + off, 16, 1024), sdesc_sw128(q_addr + kk * 2048, BM * 128, 1024),
                  idesc_kv, (step > 0 || kk > 0));
           mma_ss(tmem + kColDPT, sdesc_sw128(ds_addr + kk * 2048, 128 * 128, 1024),
                  sdesc_sw128(k_addr + kk * 2048, BN * 128, 1024), idesc_dq, kk > 0);
         }
-        // every MMA of the step is done: dQ_i may leave TMEM and Q_i/dO_i are free
+        // every MMA of the step is done: dQ_i may leave TMEM, Q_i/dO_i are free,
+        // and the dS^T tile may be rewritten
         mma_commit(&s.dkq_done);
+        if (!(ok = next_s(step + 1, true))) break;
       }
       mma_commit(&s.drain);
       mbar_wait_drain(&s.drain, 0, p.wait_limit);
@@ -483,12 +494,43 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t ds_row = smem_u32(s.ds) + r * 128;
     bool ok = true;
+    uint32_t keep[32];  // this thread's P^T of the step (bf16 pairs), reused by the dS^T phase
+    // dQ_t (this thread: query row r, columns [grp D/2, grp D/2 + D/2)) from TMEM
+    // into step t's own Q_t / dO_t buffers (box c: columns 32c .. 32c+31, 16 KB,
+    // 128B-swizzled like the TMA map) for the producer's reduce-add
+    auto drain = [&](int t) -> bool {
+      const int st = t % NSTQ;
+      if (!__all_sync(0xffffffffu, mbar_wait(&s.dkq_done, t & 1, ab))) return false;
+      tc_fence_after();
+      uint32_t a[D / 2];
+#pragma unroll
+      for (int c = 0; c < D / 64; ++c)
+        tmem_ld32(tmem + lane_off + kColDPT + grp * (D / 2) + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&a[c * 32]));
+      tmem_wait_ld();
+      reg_fence(a);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.tmem_free);
+#pragma unroll
+      for (int cl = 0; cl < D / 64; ++cl) {
+        const int c = grp * (D / 64) + cl;
+        const uint32_t row = smem_u32(dq_box(st, c)) + r * 128;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int e = cl * 32 + 4 * u;
+          st_shared_v4(row + ((u ^ (r & 7)) << 4), a[e], a[e + 1], a[e + 2], a[e + 3]);
+        }
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.staged[st]);
+      return true;
+    };
     for (int step = 0; step < n_steps; ++step) {
       const int st = step % NSTQ;
       const int h = hk * G + step / per_head;
       const int i0 = (i_first + step % per_head) * BM;
-      // S^T and dP^T are in TMEM, and the previous step's MMAs have released the
-      // dS^T tile; q_full of this stage (LSE/D rows) completed before
+      // S^T is in TMEM; q_full of this stage (LSE/D rows) completed before
       ok = __all_sync(0xffffffffu, mbar_wait(&s.st_full, step & 1, ab));
       if (!ok) break;
       tc_fence_after();
@@ -503,53 +545,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t st_col = tmem + lane_off + kColST, dp_col = tmem + lane_off + kColDPT;
       if (need_mask)
         ok = bwd_p_half<true, BIAS>(grp, &s.s_read, step & 1, ab, st_col, s.nlse2[st], p.scale_log2, bcol,
-                                    neg_slope2, p.Nk, i0, len_q, kj, len_k, diag + p.win_r, p.win_l - diag, diag);
+                                    neg_slope2, p.Nk, i0, len_q, kj, len_k, diag + p.win_r, p.win_l - diag, diag, keep);
       else
         ok = bwd_p_half<false, BIAS>(grp, &s.s_read, step & 1, ab, st_col, s.nlse2[st], p.scale_log2, bcol,
-                                     neg_slope2, p.Nk, i0, len_q, kj, len_k, 0, 0, diag);
+                                     neg_slope2, p.Nk, i0, len_q, kj, len_k, 0, 0, diag, keep);
       if (!ok) break;
       tmem_wait_st();
-      if constexpr (kDvEarly) {  // P^T is in TMEM: the dV MMAs may start
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&s.pt_ready);
-      }
-      // dP^T of this step (committed after S^T)
+      // P^T is in TMEM: the dV MMAs (and the next step's scores) may start
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&s.pt_ready);
+      // dP^T of this step
       ok = __all_sync(0xffffffffu, mbar_wait(&s.dp_full, step & 1, ab));
       if (!ok) break;
       tc_fence_after();
-      bwd_ds_half(grp, st_col, dp_col, s.drow[st], ds_row, r);
+      bwd_ds_half_kept(grp, keep, dp_col, s.drow[st], ds_row, r);
       fence_proxy_async_smem();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s.ds_ready);
-      // ---- dQ_i (this thread: query row r, columns [grp D/2, grp D/2 + D/2))
-      ok = __all_sync(0xffffffffu, mbar_wait(&s.dkq_done, step & 1, ab));
-      if (!ok) break;
-      tc_fence_after();
-      uint32_t a[D / 2];
-#pragma unroll
-      for (int c = 0; c < D / 64; ++c)
-        tmem_ld32(tmem + lane_off + kColDPT + grp * (D / 2) + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&a[c * 32]));
-      tmem_wait_ld();
-      reg_fence(a);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s.tmem_free);
-      // box c (columns 32c .. 32c+31, 16 KB) at dq_box(st, c), 128B-swizzled like the TMA map
-#pragma unroll
-      for (int cl = 0; cl < D / 64; ++cl) {
-        const int c = grp * (D / 64) + cl;
-        const uint32_t row = smem_u32(dq_box(st, c)) + r * 128;
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int e = cl * 32 + 4 * u;
-          st_shared_v4(row + ((u ^ (r & 7)) << 4), a[e], a[e + 1], a[e + 2], a[e + 3]);
-        }
-      }
-      fence_proxy_async_smem();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&s.staged[st]);
+      if (!(ok = drain(step))) break;
     }
     // ---- epilogue: dV (columns [grp DV/2, grp DV/2 + DV/2)) and dK (scaled,
     // columns [grp D/2, grp D/2 + D/2)) of key row r.  The MMA warp commits

@@ -270,7 +270,8 @@ ATTN_DEVINL float ex2(float x) {
   return y;
 }
 
-// 2^x on the FMA pipe, for x <= 0 (inputs below -126 give about 2^-126).
+// 2^x on the FMA pipe, for x <= 0 (inputs below -125 give about 2^-125: the
+// clamp keeps n + exponent(p) >= -126, so the result is never subnormal).
 // Cody and Waite's range reduction: x = n + f with n = round(x) (added to
 // 1.5 * 2^23, whose low mantissa bits then hold n) and f in [-1/2, 1/2]; 2^f
 // from the degree-3 polynomial of least maximum relative error on [-1/2, 1/2],
@@ -279,7 +280,7 @@ ATTN_DEVINL float ex2(float x) {
 // exponent field by an integer add.  Lets a share of the exponentials bypass
 // the MUFU unit.
 ATTN_DEVINL float ex2_poly(float x) {
-  x = fmaxf(x, -126.f);
+  x = fmaxf(x, -125.f);
   const float t = __fadd_rn(x, 12582912.f);
   const float f = __fsub_rn(x, __fsub_rn(t, 12582912.f));
   float p = fmaf(0.0551716685295105f, f, 0.2426111251115799f);

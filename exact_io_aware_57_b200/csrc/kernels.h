@@ -141,6 +141,7 @@ int launch_fwd_naive(const TcGeom& g, __nv_bfloat16* o, float* lse, float* s_scr
 // One warp that waits on a barrier nothing arrives on, giving up after
 // limit_cycles (the shared bounded-wait failure path).
 int launch_wait_selftest(long long limit_cycles, cudaStream_t st);
+int launch_ex2_selftest(const float* x, float* y, long long n, cudaStream_t st);
 
 // Tensor-map encoding (driver entry point resolved at run time).
 int encode_tmap_bf16(CUtensorMap* map, const void* base, int rank, const uint64_t* dims,

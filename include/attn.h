@@ -318,6 +318,18 @@ int attn_device_status(void* stream);
 int attn_selftest_wait_timeout(long long limit_cycles, void* stream);
 
 /*
+ * Self-test of the FMA-pipe exponential that the tensor-core kernels use for a
+ * share of their exponentials instead of the MUFU unit: y[i] = 2^x[i] for
+ * x[i] <= 0, by Cody-Waite range reduction (x = n + f, |f| <= 1/2) and a
+ * degree-3 polynomial for 2^f of least maximum relative error (Remez fit),
+ * relative error below 7.6e-5 -- well under the 2^-9 resolution of the bf16
+ * probabilities it feeds.  Inputs below -125 (including -inf) give 2^-125 up
+ * to that error; inputs above 0 are outside its domain.  x, y: DEVICE fp32
+ * [n], caller-owned, n >= 0.  Asynchronous on `stream`.
+ */
+int attn_selftest_ex2(const float* x, float* y, long long n, void* stream);
+
+/*
  * Kernel launches issued by this library on the calling host thread since the
  * last reset (reset = 1 clears after reading).  Lets callers count the GPU
  * work of a timed region.
