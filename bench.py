@@ -606,9 +606,12 @@ def run_reference(args):
         return  # the oracle runs on rank 0's host cores only
     K, W = args.steps, args.warmup
     budget = 150.0  # seconds for the whole run
-    prefix, heads = plan_oracle_sample(max(0.05, budget / max(1, K + W)))
+    target = max(0.05, budget / max(1, K + W))
+    prefix, heads = plan_oracle_sample(target)
     for _ in range(W):
-        oracle_sample(prefix, heads, args.seed)
+        dt, _ = oracle_sample(prefix, heads, args.seed)
+        if dt > 1.2 * target:  # the short calibration underestimated: shrink (cost ~ prefix^2)
+            prefix = max(256, int(prefix * math.sqrt(target / dt)) // 128 * 128)
     t = fl = 0.0
     for _ in range(K):
         dt, f = oracle_sample(prefix, heads, args.seed)

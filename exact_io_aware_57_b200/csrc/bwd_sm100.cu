@@ -95,6 +95,7 @@ struct BwdParams {
   __nv_bfloat16* dv;
   const float* bias;
   long long bias_bstride;
+  int batch_inner;  // grid (batch, key tile, KV head): the batch elements sharing one bias run together
   const float* alibi;
   const int* cu_q;  // packed sequences: prefix offsets (device), or null
   const int* cu_k;
@@ -264,7 +265,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // grid (key tile, KV head, batch or sequence): the key tiles of one head run
   // side by side and share its Q / dO tiles in L2 (a heaviest-first order across
   // heads measured 13 % slower on the causal workload)
-  const int n_tile = blockIdx.x, hk = blockIdx.y, zz = blockIdx.z;
+  const int n_tile = p.batch_inner ? blockIdx.y : blockIdx.x, hk = p.batch_inner ? blockIdx.z : blockIdx.y;
+  const int zz = p.batch_inner ? blockIdx.x : blockIdx.z;
   const int n0 = n_tile * BN;
   // dense: batch element b; packed: sequence blockIdx.z at rows q_off / k_off of batch 0
   int b = zz, q_off = 0, k_off = 0, len_q = p.Nq, len_k = p.Nk;
@@ -659,7 +661,9 @@ int launch_main_t(const TcGeom& g, const CUtensorMap& mq, const CUtensorMap& mk,
   auto kern = bwd_main_kernel<D, DV, BIAS>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return ATTN_ERR_CUDA;
-  dim3 grid(((g.cu_q ? g.max_nk : g.Nk) + BN - 1) / BN, g.Hkv, p.n_z);
+  const unsigned n_tiles = ((g.cu_q ? g.max_nk : g.Nk) + BN - 1) / BN;
+  const dim3 grid = p.batch_inner ? dim3(p.n_z, n_tiles, g.Hkv) : dim3(n_tiles, g.Hkv, p.n_z);
+  if (grid.y > 65535 || grid.z > 65535) return ATTN_ERR_UNSUPPORTED;
   record_kernel_event(ATTN_KERNEL_BWD, 0, st);
   kern<<<grid, kThreads, smem, st>>>(mq, mk, mv, mdo, mdq, p);
   record_kernel_event(ATTN_KERNEL_BWD, 1, st);
@@ -721,6 +725,9 @@ int launch_bwd_sm100(const TcGeom& g, const __nv_bfloat16* o, const float* lse, 
   p.dv = dv;
   p.bias = g.bias;
   p.bias_bstride = g.bias_bstride;
+  // a dense bias shared by the batch elements: run them side by side so that
+  // they read each bias tile from L2 instead of each from memory
+  p.batch_inner = g.bias && g.bias_bstride == 0 && !g.cu_q && g.B > 1;
   p.alibi = g.alibi;
   p.cu_q = g.cu_q;
   p.cu_k = g.cu_k;

@@ -17,6 +17,10 @@ int fwd_params(const TcGeom& g, __nv_bfloat16* o, float* lse, const SplitKV* spl
   p.lse = lse;
   p.bias = g.bias;
   p.bias_bstride = g.bias_bstride;
+  p.bias_vec4 = g.bias && (reinterpret_cast<uintptr_t>(g.bias) % 16 == 0) && g.Nk % 4 == 0 && g.bias_bstride % 4 == 0;
+  // a bias shared by the batch elements: run them side by side so that they
+  // read each bias tile from L2 instead of each from memory
+  p.batch_inner = g.bias && g.bias_bstride == 0 && !g.cu_q && g.B > 1 && !split;
   p.alibi = g.alibi;
   p.cu_q = g.cu_q;
   p.cu_k = g.cu_k;

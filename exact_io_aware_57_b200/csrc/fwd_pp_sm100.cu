@@ -138,9 +138,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   // ---- work: heavy (late) row blocks first under causal masking
-  const int blk = p.causal ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x;
-  const int h = blockIdx.y;
-  const int z = PARTIAL ? (int)blockIdx.z / p.num_splits : (int)blockIdx.z;
+  // grid (row block, head, batch [x split]), or (batch, row block, head) when
+  // the batch elements share a dense bias
+  const bool bi = !PARTIAL && p.batch_inner;
+  const int nblk = bi ? (int)gridDim.y : (int)gridDim.x, blk_raw = bi ? (int)blockIdx.y : (int)blockIdx.x;
+  const int blk = p.causal ? nblk - 1 - blk_raw : blk_raw;
+  const int h = bi ? (int)blockIdx.z : (int)blockIdx.y;
+  const int z = bi ? (int)blockIdx.x : PARTIAL ? (int)blockIdx.z / p.num_splits : (int)blockIdx.z;
   const int split = PARTIAL ? (int)blockIdx.z % p.num_splits : 0;
   int q_off = 0, len_q = p.Nq, k_off = 0, len_k = p.Nk, bidx = z;
   if (p.cu_q) {
@@ -331,11 +335,38 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_ld32(col_s + c * 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[c * 32]));
       tmem_wait_ld();
       reg_fence(sr);
-      if constexpr (!FAST) {
+      if constexpr (BIAS == kBiasDense) {
+        // the next tile's bias row into L2 while this tile is worked on
+        // (four 128-byte lines, clamped inside the row)
+        if (step + 1 < my.n) {
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(brow + min(kbase + BN + 32 * u, len_k - 1)));
+        }
+      }
+      if constexpr (BIAS == kBiasDense) {
+        // whole tiles of 16-byte aligned rows as float4 (a lane reads its own
+        // row, so a warp load touches 32 rows: 16 bytes each instead of 4)
+        if (p.bias_vec4 && kbase + BN <= len_k) {  // warp-uniform
+          const float4* b4 = reinterpret_cast<const float4*>(brow + kbase);
+#pragma unroll
+          for (int c4 = 0; c4 < BN / 4; ++c4) {
+            const float4 bv = __ldg(b4 + c4);
+            const float bb[4] = {bv.x, bv.y, bv.z, bv.w};
+#pragma unroll
+            for (int u = 0; u < 4; ++u)
+              sr[4 * c4 + u] = __float_as_uint(fmaf(bb[u], kLog2e, __uint_as_float(sr[4 * c4 + u]) * p.scale_log2));
+          }
+        } else {
+#pragma unroll
+          for (int c = 0; c < BN; ++c)
+            sr[c] = __float_as_uint(
+                fmaf(__ldg(brow + min(kbase + c, len_k - 1)), kLog2e, __uint_as_float(sr[c]) * p.scale_log2));
+        }
+      } else if constexpr (!FAST) {
 #pragma unroll
         for (int c = 0; c < BN; ++c) {
           float x = __uint_as_float(sr[c]) * p.scale_log2;
-          if constexpr (BIAS == kBiasDense) x = fmaf(__ldg(brow + min(kbase + c, len_k - 1)), kLog2e, x);
           if constexpr (BIAS == kBiasAlibi) x = fmaf(neg_slope2, fabsf(static_cast<float>(kbase + c - i - diag)), x);
           sr[c] = __float_as_uint(x);
         }
@@ -487,7 +518,9 @@ int launch_pp_t(const TcGeom& g, const CUtensorMap& mq, const CUtensorMap& mk, c
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return ATTN_ERR_CUDA;
   const int max_nq = g.cu_q ? g.max_nq : g.Nq;
-  dim3 grid((max_nq + 2 * BM - 1) / (2 * BM), g.Hq, (g.cu_q ? g.num_seqs : g.B) * p.num_splits);
+  const unsigned nblk = (max_nq + 2 * BM - 1) / (2 * BM), nz = (g.cu_q ? g.num_seqs : g.B) * p.num_splits;
+  const dim3 grid = (!PARTIAL && p.batch_inner) ? dim3(nz, nblk, g.Hq) : dim3(nblk, g.Hq, nz);
+  if (grid.y > 65535 || grid.z > 65535) return ATTN_ERR_UNSUPPORTED;
   record_kernel_event(ATTN_KERNEL_FWD, 0, st);
   kern<<<grid, kThreads, smem, st>>>(mq, mk, mv, p);
   record_kernel_event(ATTN_KERNEL_FWD, 1, st);

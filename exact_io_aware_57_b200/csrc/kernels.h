@@ -87,6 +87,8 @@ struct FwdParams {
   float* lse;
   const float* bias;
   long long bias_bstride;
+  int bias_vec4;       // dense bias rows 16-byte aligned: whole key tiles read as float4
+  int batch_inner;     // grid (batch, row block, head): the batch elements sharing one bias run together
   const float* alibi;  // per-query-head slopes (BIAS == kBiasAlibi)
   const int* cu_q;
   const int* cu_k;

@@ -50,6 +50,12 @@ def test_bwd_bf16_bias_gqa(orc):
     check_bwd(orc, 2, 4, 2, 257, 257, 128, True, bias=True)
 
 
+def test_bwd_bf16_bias_shared_three_batches(orc):
+    """A bias shared by three batch elements: their CTAs run side by side
+    (batch-innermost grid); rows of 388 keys with a ragged last tile."""
+    check_bwd(orc, 3, 4, 2, 388, 388, 128, True, bias=True)
+
+
 def test_fwd_bwd_full_size_causal_d128(orc):
     """The causal workload at full size (batch 2, 32 heads, N=8192, d=128, Q/K std 3),
     launched exactly as the benchmark launches it: sampled forward rows on three

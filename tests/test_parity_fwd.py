@@ -48,6 +48,33 @@ def test_fwd_bf16_bias_noncausal_d64(orc):
     check_fwd(orc, 1, 2, 1, 190, 190, 64, False, bias=True)
 
 
+@pytest.mark.parametrize("per_batch", [False, True])
+@pytest.mark.parametrize("d", [64, 128])
+def test_fwd_bf16_bias_rows_of_vectors(orc, per_batch, d):
+    """Rows of 388 keys (a multiple of 4: whole key tiles are read as 16-byte
+    vectors) with a ragged last tile (read element by element); with a shared
+    bias the three batch elements run side by side, with a per-batch one in the
+    usual order."""
+    check_fwd(orc, 3, 4, 2, 388, 388, d, True, bias=True, per_batch_bias=per_batch)
+
+
+def test_fwd_bf16_bias_unaligned_view(orc):
+    """A bias view that starts 4 bytes into its allocation: the rows are not
+    16-byte aligned, so every tile is read element by element."""
+    from parity import gpu_fwd
+
+    inp = synth.make_dense(2, 2, 2, 256, 256, 128, seed=3, with_dout=False)
+    b = synth.alibi_like_bias(2, 256, 256)
+    store = torch.empty(b.numel() + 1, dtype=torch.float32, device="cuda")
+    view = store[1:].view(b.shape)
+    view.copy_(b.cuda())
+    assert view.data_ptr() % 16 != 0
+    o, lse = gpu_fwd(inp, True, bias=view)
+    o_ref, lse_ref = orc.fwd(inp.q, inp.k, inp.v, bias=b, causal=True)
+    assert max_abs(o.double().numpy(), o_ref) <= TOL_O_BF16
+    assert max_abs(lse.double().numpy(), lse_ref) <= TOL_LSE_BF16
+
+
 def test_fwd_f32_single_head(orc):
     """The fp32 workload: batch 1, 1 head, N=128, d=64, non-causal."""
     check_fwd(orc, 1, 1, 1, 128, 128, 64, False, dtype=torch.float32)
