@@ -5,7 +5,7 @@ import pytest
 import torch
 
 from exact_io_aware_57_b200 import synth
-from parity import (TOL_GRAD_BF16, TOL_LSE_BF16, TOL_O_BF16, check_bwd, check_fwd_sampled, gpu_fwd_bwd,
+from parity import (TOL_GRAD_BF16, TOL_LSE_BF16, TOL_O_BF16, check_bwd, check_fwd_sampled, gpu_fwd_bwd, max_abs,
                     rel_fro, sample_rows)
 
 pytestmark = [pytest.mark.gpu,
@@ -71,3 +71,21 @@ def test_fwd_bwd_full_size_causal_d128(orc):
     for name, a, r in (("dq", sl(dq), dq_r), ("dk", sl(dk), dk_r), ("dv", sl(dv), dv_r)):
         e = rel_fro(a.double().numpy(), r)
         assert e <= TOL_GRAD_BF16, f"{name} rel Frobenius {e:.3e}"
+
+
+def test_bwd_bf16_per_batch_bias(orc):
+    """A bias of its own per batch element [B, Hq, N, N]: the usual grid order."""
+    inp = synth.make_dense(2, 4, 2, 300, 300, 128, seed=5)
+    b = synth.alibi_like_bias(4, 300, 300)
+    b = torch.stack([b, 0.5 * b])
+    _, _, dq, dk, dv = gpu_fwd_bwd(inp, True, bias=b)
+    dq_r, dk_r, dv_r = orc.bwd(inp.q, inp.k, inp.v, inp.dout, bias=b, causal=True)
+    for name, a, r in (("dq", dq, dq_r), ("dk", dk, dk_r), ("dv", dv, dv_r)):
+        e = rel_fro(a.double().numpy(), r)
+        assert e <= TOL_GRAD_BF16, f"{name} rel Frobenius {e:.3e}"
+
+
+def test_bwd_bf16_shared_bias_noncausal(orc):
+    """A shared dense bias over three batch elements (batch-innermost grid),
+    non-causal: every key tile of every step is unmasked except the ragged one."""
+    check_bwd(orc, 3, 4, 2, 388, 388, 128, False, bias=True)
