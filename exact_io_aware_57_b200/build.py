@@ -15,7 +15,7 @@ PKG = Path(__file__).resolve().parent
 CSRC = PKG / "csrc"
 OBJ = PKG / "_build"
 LIB = PKG / "libattn.so"
-SOURCES = ["attn_api.cu", "kernels_f32.cu", "fwd_launch.cu", "fwd_pp_sm100.cu", "bwd_sm100.cu", "naive.cu", "bwd_noalloc.cu", "merge.cu", "selftest.cu", "quant_fp8.cu"]
+SOURCES = ["attn_api.cu", "kernels_f32.cu", "fwd_launch.cu", "fwd_pp_sm100.cu", "fwd_db_sm100.cu", "bwd_sm100.cu", "naive.cu", "bwd_noalloc.cu", "merge.cu", "selftest.cu", "quant_fp8.cu"]
 HEADERS = ["common.cuh", "kernels.h"]
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")
 FLAGS = ["-std=c++17", "-O3", "-lineinfo", "-Xcompiler", "-fPIC", "-gencode", "arch=compute_100a,code=sm_100a",

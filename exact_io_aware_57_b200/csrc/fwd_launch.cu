@@ -76,8 +76,19 @@ int launch_fwd_sm100(const TcGeom& g, __nv_bfloat16* o, float* lse, cudaStream_t
   // FAST: no bias and a positive scale, so the row max can be taken on raw scores
   const bool fast = !g.bias && !g.alibi && g.scale > 0.f;
   if (dv != g.D && (split || g.bias || g.alibi)) return ATTN_ERR_UNSUPPORTED;
-  return launch_fwd_pp(g, mq, mk, mv, p, g.bias ? kBiasDense : g.alibi ? kBiasAlibi : kBiasNone, fast,
-                       split != nullptr, st);
+  const int bias_kind = g.bias ? kBiasDense : g.alibi ? kBiasAlibi : kBiasNone;
+  if (bias_kind == kBiasDense && !split && !g.cu_q) {
+    // dense bias: the 64-key kernel (K and V maps with 64-row boxes)
+    const uint32_t box64[4] = {64, 1, 64, 1};
+    const uint64_t dims[4] = {(uint64_t)g.D, (uint64_t)g.Hkv, (uint64_t)g.Nk, (uint64_t)B};
+    const uint64_t str[3] = {(uint64_t)g.D * 2, (uint64_t)g.Hkv * g.D * 2, (uint64_t)g.Nk * g.Hkv * g.D * 2};
+    if (encode_tmap_bf16(&mk, g.k, 4, dims, str, box64) != ATTN_OK) return ATTN_ERR_CUDA;
+    const uint64_t dv_dims[4] = {(uint64_t)dv, (uint64_t)g.Hkv, (uint64_t)g.Nk, (uint64_t)B};
+    const uint64_t dv_str[3] = {(uint64_t)dv * 2, (uint64_t)g.Hkv * dv * 2, (uint64_t)g.Nk * g.Hkv * dv * 2};
+    if (encode_tmap_bf16(&mv, g.v, 4, dv_dims, dv_str, box64) != ATTN_OK) return ATTN_ERR_CUDA;
+    return launch_fwd_db(g, mq, mk, mv, p, st);
+  }
+  return launch_fwd_pp(g, mq, mk, mv, p, bias_kind, fast, split != nullptr, st);
 }
 
 }  // namespace attn

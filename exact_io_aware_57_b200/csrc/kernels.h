@@ -114,6 +114,10 @@ struct FwdParams {
 // partials to p.o_part / p.lse_part.
 int launch_fwd_pp(const TcGeom& g, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                   const FwdParams& p, int bias_kind, bool fast, bool partial, cudaStream_t st);
+// Forward with a dense bias: 64-key tiles and double-buffered scores
+// (fwd_db_sm100.cu); K and V maps with 64-row boxes.  Dense batches, d = d_v.
+int launch_fwd_db(const TcGeom& g, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                  const FwdParams& p, cudaStream_t st);
 // The same kernel with e4m3 Q/K tiles (maps over the quantised tensors).
 int launch_fwd_pp_fp8(const TcGeom& g, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                       const FwdParams& p, cudaStream_t st);
