@@ -262,13 +262,21 @@ __global__ void __launch_bounds__(kThreads, 1)
   Smem& s = *reinterpret_cast<Smem*>(smem_raw);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // grid (key tile, KV head, batch or sequence): the key tiles of one head run
-  // side by side and share its Q / dO tiles in L2 (a heaviest-first order across
-  // heads measured 13 % slower on the causal workload)
-  const int n_tile = p.batch_inner ? blockIdx.y : blockIdx.x, hk = p.batch_inner ? blockIdx.z : blockIdx.y;
-  const int zz = p.batch_inner ? blockIdx.x : blockIdx.z;
+  // grid (key tile, KV head, batch or sequence): the key tiles of groups of four
+  // (batch, head) pairs are interleaved (grouped_unit), so that the heavy causal
+  // tiles start early while the CTAs running at one time still share a few
+  // heads' Q / dO tiles in L2 (a heaviest-first order across all heads measured
+  // 13 % slower on the causal workload)
+  int n_tile, hk, zz;
+  if (p.batch_inner) {
+    n_tile = blockIdx.y, hk = blockIdx.z, zz = blockIdx.x;
+  } else {
+    int u;
+    grouped_unit((int)gridDim.x, (int)(gridDim.y * gridDim.z), 4, n_tile, u);
+    hk = u % p.Hkv, zz = u / p.Hkv;
+  }
   const int n0 = n_tile * BN;
-  // dense: batch element b; packed: sequence blockIdx.z at rows q_off / k_off of batch 0
+  // dense: batch element b; packed: sequence zz at rows q_off / k_off of batch 0
   int b = zz, q_off = 0, k_off = 0, len_q = p.Nq, len_k = p.Nk;
   if (p.cu_q) {
     // invalid offsets: reported in the status word, nothing read or written

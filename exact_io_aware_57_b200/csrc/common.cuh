@@ -100,6 +100,21 @@ ATTN_DEVINL bool packed_seq(const int* cu, int z, int total, int max_len, int* s
   return true;
 }
 
+// Work unit of this CTA in a launch of nr x nu units (rank r of the row or key
+// tiles, u = the (batch, head) pair).  CTAs start roughly in launch order, so
+// the units are listed by groups of `gs` consecutive u: every u of the group at
+// rank 0, then every u at rank 1, and so on.  With rank 0 the heaviest, the
+// heavy units of all groups but the last start early and the last CTAs to start
+// are light (a short tail), while the CTAs running at one time span few heads
+// and share their K/V (or Q/dO) tiles in L2.
+ATTN_DEVINL void grouped_unit(int nr, int nu, int gs, int& r, int& u) {
+  const int i = (int)(blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z));
+  const int g = i / (gs * nr), base = g * gs, gn = min(gs, nu - base);
+  const int rem = i - g * gs * nr;
+  r = rem / gn;
+  u = base + rem % gn;
+}
+
 // ------------------------------------------------------------------------- TMA
 ATTN_DEVINL void tma_prefetch_desc(const CUtensorMap* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");

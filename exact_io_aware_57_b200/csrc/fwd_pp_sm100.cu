@@ -138,13 +138,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   // ---- work: heavy (late) row blocks first under causal masking
-  // grid (row block, head, batch [x split]), or (batch, row block, head) when
-  // the batch elements share a dense bias
+  // grid (row block, head, batch [x split]); the row blocks of groups of eight
+  // (batch, head) pairs are interleaved (grouped_unit), or, when the batch
+  // elements share a dense bias, (batch, row block, head)
   const bool bi = !PARTIAL && p.batch_inner;
-  const int nblk = bi ? (int)gridDim.y : (int)gridDim.x, blk_raw = bi ? (int)blockIdx.y : (int)blockIdx.x;
+  const int nblk = bi ? (int)gridDim.y : (int)gridDim.x;
+  int blk_raw, h, z;
+  if (PARTIAL) {
+    blk_raw = blockIdx.x, h = blockIdx.y, z = blockIdx.z / p.num_splits;
+  } else if (bi) {
+    blk_raw = blockIdx.y, h = blockIdx.z, z = blockIdx.x;
+  } else {
+    int u;
+    grouped_unit(nblk, (int)(gridDim.y * gridDim.z), 8, blk_raw, u);
+    h = u % p.Hq, z = u / p.Hq;
+  }
   const int blk = p.causal ? nblk - 1 - blk_raw : blk_raw;
-  const int h = bi ? (int)blockIdx.z : (int)blockIdx.y;
-  const int z = bi ? (int)blockIdx.x : PARTIAL ? (int)blockIdx.z / p.num_splits : (int)blockIdx.z;
   const int split = PARTIAL ? (int)blockIdx.z % p.num_splits : 0;
   int q_off = 0, len_q = p.Nq, k_off = 0, len_k = p.Nk, bidx = z;
   if (p.cu_q) {
