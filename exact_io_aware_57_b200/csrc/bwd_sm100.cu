@@ -29,18 +29,21 @@
 // Per step (query head h, query tile i):
 //   MMA   dP^T = V_j dO_i^T once the previous dQ has left TMEM (S^T of this step
 //         was issued earlier, see below)
-//   WGs   P^T = 2^(scale log2e S^T + log2e B^T - log2e LSE) -> TMEM (bf16),
-//         overlapping the dP^T MMAs; P^T also stays in registers for dS^T;
+//   WGs   P^T = 2^(scale log2e S^T + log2e B^T - log2e LSE) -> TMEM (bf16,
+//         each group over its own half of the S^T columns), overlapping the
+//         dP^T MMAs; P^T also stays in registers for dS^T;
 //         dS^T = P^T o (dP^T - D) -> shared memory (bf16, 128B-swizzled)
 //   MMA   dV += P^T dO_i (P^T from TMEM) once P^T is there, overlapping dS^T;
 //         S^T of the next step = K_j Q_{i+1}^T as soon as Q_{i+1} has arrived
 //         (the scores columns are free once P^T has been read out), so the
-//         elementwise groups find the next scores ready; then dK += dS^T Q_i
-//         and dQ_i = dS K_j, round-robin
-//   WGs   dQ_i -> the step's own Q_i/dO_i buffers (free once its MMAs are done);
-//         the producer adds them into the fp32 accumulator with TMA bulk
-//         reductions and refills the buffers only after those have read them,
-//         so the reduction overlaps the next step instead of holding it up.
+//         elementwise groups find the next scores ready; then dQ_i = dS K_j
+//         and, after it, dK += dS^T Q_i
+//   WGs   dQ_i -> the step's own Q_i/dO_i buffers as soon as the dQ MMAs are
+//         done (the Q_i half only after dK has read Q_i); the next dP^T may
+//         start in its columns while dK runs.  The producer adds the staged
+//         tile into the fp32 accumulator with TMA bulk reductions and refills
+//         the buffers only after those have read them, so the reduction
+//         overlaps the next step instead of holding it up.
 #include <algorithm>
 
 #include "common.cuh"
@@ -82,7 +85,7 @@ struct BwdSmem {
   alignas(16) float nlse2[NSTQ][BM];        // -log2(e) * LSE of the step's query rows (-inf: no key)
   alignas(16) float drow[NSTQ][BM];         // D_i of the step's query rows
   uint64_t kv_full, q_full[NSTQ], staged[NSTQ];
-  uint64_t st_full, dp_full, s_read, pt_ready, ds_ready, dkq_done, tmem_free, drain;
+  uint64_t st_full, dp_full, pt_ready, ds_ready, dq_done, dkq_done, tmem_free, drain;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -169,19 +172,21 @@ ATTN_DEVINL void p_chunk(int c, const uint32_t (&sr)[32], uint32_t st_col, const
     pk[2 * e4] = pack_bf16(pv[0], pv[1]);
     pk[2 * e4 + 1] = pack_bf16(pv[2], pv[3]);
   }
-  tmem_st16(st_col + c * 16, pk);  // columns [16c, 16c+16): S^T there is already read
+  // chunk c (32 queries, 16 columns of bf16 pairs) over S^T columns this thread
+  // has already read: [16c, 16c+16) for group 0's chunks 0, 1 and [16c+32,
+  // 16c+48) for group 1's chunks 2, 3, so neither group writes over the
+  // other's scores
+  tmem_st16(st_col + c * 16 + (c & 2) * 16, pk);
 }
 
-// Group g's half of phase A: queries [64g, 64g+64), chunks 2g and 2g+1.  The
-// P^T of group 1 lands on S^T columns [32, 64), which group 0 reads: group 0's
-// warps arrive on `s_read` once their loads are complete and group 1 waits for
-// that phase (bounded) before it stores.  Returns false if that wait gave up.
+// Group g's half of phase A: queries [64g, 64g+64), chunks 2g and 2g+1, read
+// from S^T columns [64g, 64g+64) and written back as P^T into the first half of
+// the same columns (p_chunk), so the two groups need not wait for each other.
 // keep: this thread's P^T as bf16 pairs (chunk 2g in [0,16), chunk 2g+1 in [16,32)).
 template <bool MASK, int BIAS>
-ATTN_DEVINL bool bwd_p_half(int grp, uint64_t* s_read, uint32_t parity, const Abort& ab, uint32_t st_col,
-                            const float* nlse2, float scale_log2, const float* bcol, float neg_slope2, int nk, int i0,
-                            int len_q, int kj, int len_k, int lo_off, int hi_off, int bias_diag,
-                            uint32_t (&keep)[32]) {
+ATTN_DEVINL void bwd_p_half(int grp, uint32_t st_col, const float* nlse2, float scale_log2, const float* bcol,
+                            float neg_slope2, int nk, int i0, int len_q, int kj, int len_k, int lo_off, int hi_off,
+                            int bias_diag, uint32_t (&keep)[32]) {
   const int c0 = 2 * grp;
   uint32_t ra[32], rb[32];
   tmem_ld32(st_col + c0 * 32, ra);
@@ -189,19 +194,10 @@ ATTN_DEVINL bool bwd_p_half(int grp, uint64_t* s_read, uint32_t parity, const Ab
   tmem_wait_ld();
   reg_fence(ra);
   reg_fence(rb);
-  if (grp == 0) {
-    tc_fence_before();
-    __syncwarp();
-    if ((threadIdx.x & 31) == 0) mbar_arrive(s_read);
-  } else {
-    if (!__all_sync(0xffffffffu, mbar_wait(s_read, parity, ab))) return false;
-    tc_fence_after();
-  }
   p_chunk<MASK, BIAS>(c0, ra, st_col, nlse2, scale_log2, bcol, neg_slope2, nk, i0, len_q, kj, len_k, lo_off, hi_off,
                       bias_diag, *reinterpret_cast<uint32_t(*)[16]>(&keep[0]));
   p_chunk<MASK, BIAS>(c0 + 1, rb, st_col, nlse2, scale_log2, bcol, neg_slope2, nk, i0, len_q, kj, len_k, lo_off,
                       hi_off, bias_diag, *reinterpret_cast<uint32_t(*)[16]>(&keep[16]));
-  return true;
 }
 
 // Phase B -- dS^T = P^T (dP^T - D) from the bf16 P^T and dP^T, into the
@@ -308,9 +304,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     mbar_init(&s.st_full, 1);
     mbar_init(&s.dp_full, 1);
-    mbar_init(&s.s_read, 4);
     mbar_init(&s.ds_ready, 8);
     mbar_init(&s.pt_ready, 8);
+    mbar_init(&s.dq_done, 1);
     mbar_init(&s.dkq_done, 1);
     mbar_init(&s.tmem_free, 8);
     mbar_init(&s.drain, 1);
@@ -470,25 +466,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!(ok = mbar_wait(&s.pt_ready, step & 1, ab))) break;
         tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < BM / 16; ++kk)
-          mma_ts(tmem + kColDV, tmem + kColST + kk * 8, sdesc_sw128(do_addr + kk * 2048, BM * 128, 1024), idesc_dv,
-                 (step > 0 || kk > 0));
+        for (int kk = 0; kk < BM / 16; ++kk)  // queries [16kk, 16kk+16): columns kk*8 (+32 for group 1's half)
+          mma_ts(tmem + kColDV, tmem + kColST + kk * 8 + (kk >= 4 ? 32 : 0),
+                 sdesc_sw128(do_addr + kk * 2048, BM * 128, 1024), idesc_dv, (step > 0 || kk > 0));
         if (!(ok = next_s(step + 1, false))) break;
-        // dK += dS^T Q_i and dQ_i = dS K_j (the dS^T tile read MN-major) once
-        // dS^T is in shared memory, round-robin
+        // dQ_i = dS K_j (the dS^T tile read MN-major), then dK += dS^T Q_i, once
+        // dS^T is in shared memory
         if (!(ok = mbar_wait(&s.ds_ready, step & 1, ab))) break;
         if (!(ok = next_s(step + 1, false))) break;
         tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < BM / 16; ++kk)
+          mma_ss(tmem + kColDPT, sdesc_sw128(ds_addr + kk * 2048, 128 * 128, 1024),
+                 sdesc_sw128(k_addr + kk * 2048, BN * 128, 1024), idesc_dq, kk > 0);
+        // dQ_i may leave TMEM, and dO_i (last read by dV) is free
+        mma_commit(&s.dq_done);
 #pragma unroll
         for (int kk = 0; kk < BM / 16; ++kk) {
           const uint32_t off = (kk >> 2) * (128 * 128) + (kk & 3) * 32;
           mma_ss(tmem + kColDK, sdesc_sw128(ds_addr + off, 16, 1024), sdesc_sw128(q_addr + kk * 2048, BM * 128, 1024),
                  idesc_kv, (step > 0 || kk > 0));
-          mma_ss(tmem + kColDPT, sdesc_sw128(ds_addr + kk * 2048, 128 * 128, 1024),
-                 sdesc_sw128(k_addr + kk * 2048, BN * 128, 1024), idesc_dq, kk > 0);
         }
-        // every MMA of the step is done: dQ_i may leave TMEM, Q_i/dO_i are free,
-        // and the dS^T tile may be rewritten
+        // every MMA of the step is done: Q_i is free, and the dS^T tile may be
+        // rewritten
         mma_commit(&s.dkq_done);
         if (!(ok = next_s(step + 1, true))) break;
       }
@@ -508,9 +508,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     // dQ_t (this thread: query row r, columns [grp D/2, grp D/2 + D/2)) from TMEM
     // into step t's own Q_t / dO_t buffers (box c: columns 32c .. 32c+31, 16 KB,
     // 128B-swizzled like the TMA map) for the producer's reduce-add
+    // Group 0's boxes are exactly the Q_t buffer, which dK (issued after dQ)
+    // still reads: that group waits for dK before it stores; group 1's boxes
+    // (the dO_t buffer, and the extra buffer when D > DV) are free once dQ is.
+    // The next dS^T tile is written only after the next dP^T, whose commit
+    // follows this step's dK.
     auto drain = [&](int t) -> bool {
       const int st = t % NSTQ;
-      if (!__all_sync(0xffffffffu, mbar_wait(&s.dkq_done, t & 1, ab))) return false;
+      if (!__all_sync(0xffffffffu, mbar_wait(&s.dq_done, t & 1, ab))) return false;
       tc_fence_after();
       uint32_t a[D / 2];
 #pragma unroll
@@ -521,6 +526,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s.tmem_free);
+      if (grp == 0 && !__all_sync(0xffffffffu, mbar_wait(&s.dkq_done, t & 1, ab))) return false;
 #pragma unroll
       for (int cl = 0; cl < D / 64; ++cl) {
         const int c = grp * (D / 64) + cl;
@@ -554,12 +560,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       if constexpr (BIAS == kBiasAlibi) neg_slope2 = -__ldg(p.alibi + h) * kLog2e;
       const uint32_t st_col = tmem + lane_off + kColST, dp_col = tmem + lane_off + kColDPT;
       if (need_mask)
-        ok = bwd_p_half<true, BIAS>(grp, &s.s_read, step & 1, ab, st_col, s.nlse2[st], p.scale_log2, bcol,
-                                    neg_slope2, p.Nk, i0, len_q, kj, len_k, diag + p.win_r, p.win_l - diag, diag, keep);
+        bwd_p_half<true, BIAS>(grp, st_col, s.nlse2[st], p.scale_log2, bcol, neg_slope2, p.Nk, i0, len_q, kj, len_k,
+                               diag + p.win_r, p.win_l - diag, diag, keep);
       else
-        ok = bwd_p_half<false, BIAS>(grp, &s.s_read, step & 1, ab, st_col, s.nlse2[st], p.scale_log2, bcol,
-                                     neg_slope2, p.Nk, i0, len_q, kj, len_k, 0, 0, diag, keep);
-      if (!ok) break;
+        bwd_p_half<false, BIAS>(grp, st_col, s.nlse2[st], p.scale_log2, bcol, neg_slope2, p.Nk, i0, len_q, kj, len_k,
+                                0, 0, diag, keep);
       tmem_wait_st();
       // P^T is in TMEM: the dV MMAs (and the next step's scores) may start
       tc_fence_before();
