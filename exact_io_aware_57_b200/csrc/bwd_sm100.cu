@@ -84,7 +84,7 @@ struct BwdSmem {
   alignas(1024) uint8_t dqx[NSTQ][kXBoxes > 0 ? kXBoxes * 128 * 128 : 16];
   alignas(16) float nlse2[NSTQ][BM];        // -log2(e) * LSE of the step's query rows (-inf: no key)
   alignas(16) float drow[NSTQ][BM];         // D_i of the step's query rows
-  uint64_t kv_full, q_full[NSTQ], staged[NSTQ];
+  uint64_t kv_full, q_full[NSTQ], do_full[NSTQ], staged[NSTQ];
   uint64_t st_full, dp_full, pt_ready, ds_ready, dq_done, dkq_done, tmem_free, drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -129,6 +129,7 @@ ATTN_DEVINL void tma_reduce_add_4d(const CUtensorMap* map, const void* src, int 
 }
 ATTN_DEVINL void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 ATTN_DEVINL void bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+ATTN_DEVINL void bulk_wait_read1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
 ATTN_DEVINL void bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
 ATTN_DEVINL void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
@@ -299,7 +300,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     s.abort_flag = 0;
     mbar_init(&s.kv_full, 1);
     for (int i = 0; i < NSTQ; ++i) {
-      mbar_init(&s.q_full[i], 1 + 32);  // TMA transaction arrive + 32 producer lanes (LSE/D rows)
+      mbar_init(&s.q_full[i], 1 + 32);   // TMA transaction arrive + 32 producer lanes (LSE rows)
+      mbar_init(&s.do_full[i], 1 + 32);  // TMA transaction arrive + 32 producer lanes (D rows)
       mbar_init(&s.staged[i], 8);   // the eight elementwise warps, dQ tile staged
     }
     mbar_init(&s.st_full, 1);
@@ -328,9 +330,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) {
     // ===================================================== producer
     // Stage st of step s held the dQ tile of step s - NSTQ: before reloading
-    // it, add that tile into the accumulator and wait until the reduction has
-    // read the buffers.
-    int issued = 0, reduced = 0;
+    // it, add that tile into the accumulator.  The boxes staged in the Q buffer
+    // go first, as a bulk group of their own, so that Q_s (all the next scores
+    // need) loads as soon as the reduction has read them; dO_s loads, on a
+    // barrier of its own, once the rest has been read.
+    int issued = 0;
     auto reduce_step = [&](int t) -> bool {
       const int st = t % NSTQ;
       if (!__all_sync(0xffffffffu, mbar_wait(&s.staged[st], (t / NSTQ) & 1, ab))) return false;
@@ -338,13 +342,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int h = hk * G + t / per_head;
         const int i0 = (i_first + t % per_head) * BM;
 #pragma unroll
-        for (int c = 0; c < D / 32; ++c)
+        for (int c = 0; c < Smem::kQBoxes; ++c)
           tma_reduce_add_4d(&tm_dq, dq_box(st, c), c * 32, h, q_off + i0, b);
         bulk_commit();
-        bulk_wait_read0();
+#pragma unroll
+        for (int c = Smem::kQBoxes; c < D / 32; ++c)
+          tma_reduce_add_4d(&tm_dq, dq_box(st, c), c * 32, h, q_off + i0, b);
+        bulk_commit();
       }
       __syncwarp();
-      ++reduced;
       return true;
     };
     if (lane == 0) {
@@ -383,20 +389,25 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (step >= NSTQ && !(ok = reduce_step(step - NSTQ))) break;
       if (lane == 0) {
-        mbar_expect_tx(&s.q_full[st], Smem::kKBytes + Smem::kVBytes);
+        if (step >= NSTQ) bulk_wait_read1();  // the Q buffer's boxes have been read
+        mbar_expect_tx(&s.q_full[st], Smem::kKBytes);
 #pragma unroll
         for (int kb = 0; kb < KB; ++kb)
           tma_load_4d(s.q[st] + kb * BM * 128, &tm_q, &s.q_full[st], kb * 64, h, q_off + i0, b);
+      }
+#pragma unroll
+      for (int e = 0; e < BM / 32; ++e) s.nlse2[st][lane + 32 * e] = l2v[e];
+      mbar_arrive(&s.q_full[st]);
+      if (lane == 0) {
+        if (step >= NSTQ) bulk_wait_read0();  // and the rest
+        mbar_expect_tx(&s.do_full[st], Smem::kVBytes);
 #pragma unroll
         for (int kb = 0; kb < KBV; ++kb)
-          tma_load_4d(s.dout[st] + kb * BM * 128, &tm_do, &s.q_full[st], kb * 64, h, q_off + i0, b);
+          tma_load_4d(s.dout[st] + kb * BM * 128, &tm_do, &s.do_full[st], kb * 64, h, q_off + i0, b);
       }
 #pragma unroll
-      for (int e = 0; e < BM / 32; ++e) {
-        s.nlse2[st][lane + 32 * e] = l2v[e];
-        s.drow[st][lane + 32 * e] = drv[e];
-      }
-      mbar_arrive(&s.q_full[st]);
+      for (int e = 0; e < BM / 32; ++e) s.drow[st][lane + 32 * e] = drv[e];
+      mbar_arrive(&s.do_full[st]);
       ++issued;
     }
     // the last NSTQ dQ tiles
@@ -405,8 +416,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       bulk_wait0();  // every reduction has completed before the CTA exits
       if (s.abort_flag) {
         if (n_steps > 0) mbar_wait_drain(&s.kv_full, 0, p.wait_limit);
-        for (int j = max(0, issued - NSTQ); j < issued; ++j)
+        for (int j = max(0, issued - NSTQ); j < issued; ++j) {
           mbar_wait_drain(&s.q_full[j % NSTQ], (j / NSTQ) & 1, p.wait_limit);
+          mbar_wait_drain(&s.do_full[j % NSTQ], (j / NSTQ) & 1, p.wait_limit);
+        }
       }
     }
   } else if (warp == 1) {
@@ -454,6 +467,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t q_addr = smem_u32(s.q[st]), do_addr = smem_u32(s.dout[st]);
         // dP^T = V_j dO_i^T where dQ of the previous step was, once that has left
         if (step > 0 && !(ok = mbar_wait(&s.tmem_free, (step - 1) & 1, ab))) break;
+        if (!(ok = mbar_wait(&s.do_full[st], (step / NSTQ) & 1, ab))) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < DV / 16; ++kk) {
@@ -546,7 +560,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int st = step % NSTQ;
       const int h = hk * G + step / per_head;
       const int i0 = (i_first + step % per_head) * BM;
-      // S^T is in TMEM; q_full of this stage (LSE/D rows) completed before
+      // S^T is in TMEM; q_full of this stage (LSE rows) completed before, and
+      // do_full (D rows) before dP^T
       ok = __all_sync(0xffffffffu, mbar_wait(&s.st_full, step & 1, ab));
       if (!ok) break;
       tc_fence_after();
