@@ -36,6 +36,12 @@ def test_bwd_bf16_shapes(orc, B, Hq, Hkv, N, d, causal):
     check_bwd(orc, B, Hq, Hkv, N, N, d, causal)
 
 
+def test_bwd_bf16_ragged_head_groups(orc):
+    """Six (batch, KV head) pairs: the grid interleaves the key tiles of groups of
+    four pairs, so the last group holds two; four key tiles, the last ragged."""
+    check_bwd(orc, 3, 4, 2, 400, 400, 128, True, seed=12)
+
+
 @pytest.mark.parametrize("Nq,Nk", [(300, 500), (500, 300)])
 def test_bwd_bf16_unequal_lengths(orc, Nq, Nk):
     check_bwd(orc, 1, 2, 1, Nq, Nk, 128, True)

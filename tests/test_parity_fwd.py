@@ -33,6 +33,12 @@ def test_fwd_bf16_unequal_lengths(orc, Nq, Nk, causal):
     check_fwd(orc, 1, 2, 1, Nq, Nk, 128, causal)
 
 
+def test_fwd_bf16_ragged_head_groups(orc):
+    """Twelve (batch, head) pairs: the grid interleaves the row blocks of groups
+    of eight pairs, so the last group holds four; three row blocks, the last ragged."""
+    check_fwd(orc, 3, 4, 2, 600, 600, 128, True, seed=11)
+
+
 def test_fwd_bf16_peaked_scores(orc):
     """Q, K ~ N(0, 3^2): frequent running-max rescales (the causal fwd+bwd workload's regime)."""
     check_fwd(orc, 1, 2, 2, 1024, 1024, 128, True, sigma=3.0)
