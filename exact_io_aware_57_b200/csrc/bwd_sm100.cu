@@ -263,10 +263,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   // (batch, head) pairs are interleaved (grouped_unit), so that the heavy causal
   // tiles start early while the CTAs running at one time still share a few
   // heads' Q / dO tiles in L2 (a heaviest-first order across all heads measured
-  // 13 % slower on the causal workload)
+  // 13 % slower on the causal workload).  When the batch elements share a
+  // dense bias (grid (batch, key tile, KV head)), a group is every batch
+  // element of two KV heads, so the ones reading the same bias run side by side.
   int n_tile, hk, zz;
   if (p.batch_inner) {
-    n_tile = blockIdx.y, hk = blockIdx.z, zz = blockIdx.x;
+    const int nb = (int)gridDim.x;
+    int u;
+    grouped_unit((int)gridDim.y, nb * p.Hkv, 2 * nb, n_tile, u);
+    hk = u / nb, zz = u % nb;
   } else {
     int u;
     grouped_unit((int)gridDim.x, (int)(gridDim.y * gridDim.z), 4, n_tile, u);

@@ -113,14 +113,18 @@ __global__ void __launch_bounds__(kThreads, 1)
   Smem& s = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  // ---- work: heavy (late) row blocks first under causal masking; grid (row
-  // block, head, batch), or (batch, row block, head) when the batch elements
-  // share the bias
+  // ---- work: heavy (late) row blocks first under causal masking, the row
+  // blocks of a group of (batch, head) pairs interleaved (grouped_unit): eight
+  // heads of one batch element, or, when the batch elements share the bias
+  // (grid (batch, row block, head)), every batch element of two heads, so that
+  // the ones reading the same bias rows run side by side
   const bool bi = p.batch_inner;
-  const int nblk = bi ? (int)gridDim.y : (int)gridDim.x, blk_raw = bi ? (int)blockIdx.y : (int)blockIdx.x;
+  const int nblk = bi ? (int)gridDim.y : (int)gridDim.x, nb = bi ? (int)gridDim.x : (int)gridDim.z;
+  int blk_raw, u;
+  grouped_unit(nblk, nb * p.Hq, bi ? 2 * nb : 8, blk_raw, u);
   const int blk = p.causal ? nblk - 1 - blk_raw : blk_raw;
-  const int h = bi ? (int)blockIdx.z : (int)blockIdx.y;
-  const int bidx = bi ? (int)blockIdx.x : (int)blockIdx.z;
+  const int h = bi ? u / nb : u % p.Hq;
+  const int bidx = bi ? u % nb : u / p.Hq;
   const int q_off = 0, k_off = 0, len_q = p.Nq, len_k = p.Nk;
   const int m0 = blk * 2 * BM;
   if (m0 >= len_q) return;  // uniform: before any barrier or TMEM use

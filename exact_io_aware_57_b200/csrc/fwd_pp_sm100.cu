@@ -139,15 +139,20 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // ---- work: heavy (late) row blocks first under causal masking
   // grid (row block, head, batch [x split]); the row blocks of groups of eight
-  // (batch, head) pairs are interleaved (grouped_unit), or, when the batch
-  // elements share a dense bias, (batch, row block, head)
+  // (batch, head) pairs are interleaved (grouped_unit).  When the batch
+  // elements share a dense bias (grid (batch, row block, head)), a group is
+  // every batch element of two heads, so the ones reading the same bias rows
+  // run side by side
   const bool bi = !PARTIAL && p.batch_inner;
   const int nblk = bi ? (int)gridDim.y : (int)gridDim.x;
   int blk_raw, h, z;
   if (PARTIAL) {
     blk_raw = blockIdx.x, h = blockIdx.y, z = blockIdx.z / p.num_splits;
   } else if (bi) {
-    blk_raw = blockIdx.y, h = blockIdx.z, z = blockIdx.x;
+    const int nb = (int)gridDim.x;
+    int u;
+    grouped_unit(nblk, nb * p.Hq, 2 * nb, blk_raw, u);
+    h = u / nb, z = u % nb;
   } else {
     int u;
     grouped_unit(nblk, (int)(gridDim.y * gridDim.z), 8, blk_raw, u);
