@@ -18,6 +18,10 @@
 //   warp 8      TMEM owner + single-thread tcgen05.mma issuer
 //   warp 9      TMA producer: Q_0, Q_1 once, then K_j (two key tiles ahead) and
 //               V_j into smem rings
+//   warp 10     (BT: bias rows 16-byte aligned) TMA producer of the bias: each
+//               query tile's 128 x 64 fp32 bias block of its next key tile, into
+//               a buffer of its own that the softmax empties first thing, so the
+//               block of the next key tile is on its way while the softmax works
 //
 // TMEM (512 columns x 128 lanes x 32 bit):
 //   [128 t + 64 b, 128 t + 64 b + 64)  S_t of the key tiles with step parity b
@@ -41,6 +45,7 @@
 // it writes O / l and LSE = (m + log2 l) ln 2.  Causal and local masks apply
 // to the key tiles on the edges of a query tile's band only.
 #include <algorithm>
+#include <cstring>
 
 #include "common.cuh"
 #include "kernels.h"
@@ -51,25 +56,33 @@ namespace {
 
 constexpr int BM = 128;  // query rows per tile (two tiles per CTA)
 constexpr int KT = 64;   // keys per K/V tile
-constexpr int kThreads = 320;
-constexpr int kWarpMma = 8, kWarpLoad = 9;
+constexpr int kWarpMma = 8, kWarpLoad = 9, kWarpBias = 10;
+template <bool BT>
+constexpr int kThreadsOf = BT ? 352 : 320;
 constexpr uint32_t kTmemCols = 512;
 constexpr float kRescaleThreshold = 8.f;  // log2 units: P stays <= 256
 
-template <int D>
+// BT: each query tile's bias block (128 rows x 64 keys fp32, two 128B-swizzled
+// TMA boxes of 32 keys) is staged in shared memory.
+template <int D, bool BT>
 struct DBSmem {
   static constexpr int DV = D;
   static constexpr int kQBytes = BM * D * 2;
   static constexpr int kKBytes = KT * D * 2;
   static constexpr int kVBytes = KT * DV * 2;
-  // K/V ring depth: as many stages as fit beside the two Q tiles in ~222 KB
-  static constexpr int NST = std::min(8, (222 * 1024 - 2 * kQBytes) / (kKBytes + kVBytes));
+  static constexpr int kBiasBytes = BM * KT * 4;  // one query tile's block
+  // K/V ring depth: as many stages as fit beside the two Q tiles (and the two
+  // bias blocks) in ~222 KB (~226 KB with the bias blocks)
+  static constexpr int NST =
+      std::min(8, ((BT ? 226 : 222) * 1024 - 2 * kQBytes - (BT ? 2 * kBiasBytes : 0)) / (kKBytes + kVBytes));
   alignas(1024) uint8_t q[2][kQBytes];
   alignas(1024) uint8_t k[NST][kKBytes];
   alignas(1024) uint8_t v[NST][kVBytes];
+  alignas(1024) uint8_t bias[2][BT ? kBiasBytes : 16];
   uint64_t q_full;
   uint64_t k_full[NST], k_empty[NST], v_full[NST], v_empty[NST];
   uint64_t s_full[2][2], p_full[2][2];  // [query tile][score buffer]
+  uint64_t bias_full[2], bias_empty[2];  // BT: [query tile]
   uint64_t pv_last[2], o_done[2], drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -101,11 +114,12 @@ ATTN_DEVINL TileRange tile_range(int mt, int len_q, int diag, int win_l, int win
 
 ATTN_DEVINL bool in_range(const TileRange& r, int j) { return r.n > 0 && j >= r.jb && j < r.jb + r.n; }
 
-template <int D>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int D, bool BT>
+__global__ void __launch_bounds__(kThreadsOf<BT>, 1)
     fwd_db_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                  const __grid_constant__ CUtensorMap tm_v, const FwdParams p) {
-  using Smem = DBSmem<D>;
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_b,
+                  const FwdParams p) {
+  using Smem = DBSmem<D, BT>;
   constexpr int DV = D;
   constexpr int NST = Smem::NST;
   constexpr int KB = D / 64, KBV = DV / 64;  // 128-byte blocks per Q/K and V row
@@ -156,6 +170,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       mbar_init(&s.pv_last[t], 1);
       mbar_init(&s.o_done[t], 1);
+      mbar_init(&s.bias_full[t], 1);
+      mbar_init(&s.bias_empty[t], 4);  // the four warps of the tile's softmax
     }
     mbar_init(&s.drain, 1);
     fence_mbar_init();
@@ -211,6 +227,33 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_wait_drain(&s.k_full[i % NST], (i / NST) & 1, p.wait_limit);
         for (int i = max(0, issued_v - NST); i < issued_v; ++i)
           mbar_wait_drain(&s.v_full[i % NST], (i / NST) & 1, p.wait_limit);
+      }
+    }
+  } else if (BT && warp == kWarpBias) {
+    // ===================================================== bias producer
+    // One buffer per query tile: the block of its key tile `step` is loaded once
+    // the softmax has read the block of step - 1 out of shared memory.
+    if (lane == 0 && n_union > 0) {
+      tma_prefetch_desc(&tm_b);
+      const int row = q_off + m0, zb = p.bias_bstride ? bidx : 0;
+      int issued[2] = {0, 0};
+      bool ok = true;
+      for (int step = 0; ok && step < max(rg[0].n, rg[1].n); ++step) {
+        for (int t = 0; t < 2; ++t) {
+          if (step >= rg[t].n) continue;
+          if (step > 0 && !(ok = mbar_wait(&s.bias_empty[t], (step - 1) & 1, ab))) break;
+          mbar_expect_tx(&s.bias_full[t], Smem::kBiasBytes);
+          const int kb = k_off + (rg[t].jb + step) * KT;  // a multiple of 64 keys: 16-byte aligned
+#pragma unroll
+          for (int half = 0; half < 2; ++half)
+            tma_load_4d(s.bias[t] + half * (BM * 128), &tm_b, &s.bias_full[t], kb + 32 * half, row + t * BM, h, zb);
+          ++issued[t];
+        }
+      }
+      if (s.abort_flag) {
+        // at most one block per buffer is in flight: the last one issued
+        for (int t = 0; t < 2; ++t)
+          if (issued[t] > 0) mbar_wait_drain(&s.bias_full[t], (issued[t] - 1) & 1, p.wait_limit);
       }
     }
   } else if (warp == kWarpMma) {
@@ -302,7 +345,30 @@ __global__ void __launch_bounds__(kThreads, 1)
       tmem_ld32(col_s + 32, *reinterpret_cast<uint32_t(*)[32]>(&sr[32]));
       tmem_wait_ld();
       reg_fence(sr);
-      {
+      if constexpr (BT) {
+        // this row of the staged block: 16-byte chunk c of each 32-key box sits
+        // at chunk c ^ (r & 7) of the row (128-byte swizzle), so the 32 rows of
+        // a warp spread over all banks; then the buffer goes back to the producer
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(&s.bias_full[t], step & 1, ab)))) break;
+        const uint32_t brow_s = smem_u32(s.bias[t]) + r * 128;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            float bb[4];
+            asm volatile("ld.shared.v4.f32 {%0,%1,%2,%3}, [%4];"
+                         : "=f"(bb[0]), "=f"(bb[1]), "=f"(bb[2]), "=f"(bb[3])
+                         : "r"(brow_s + half * (BM * 128) + ((c ^ (r & 7)) << 4)));
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int key = 32 * half + 4 * c + e;
+              sr[key] = __float_as_uint(fmaf(bb[e], kLog2e, __uint_as_float(sr[key]) * sc2));
+            }
+          }
+        }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&s.bias_empty[t]);
+      } else {
         // the next key tile's bias row into L2 while this one is worked on (two
         // 128-byte lines, clamped inside the row); whole tiles of 16-byte
         // aligned rows as float4 (a lane reads its own row)
@@ -431,19 +497,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
-template <int D>
+template <int D, bool BT>
 int launch_db_t(const TcGeom& g, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
-                const FwdParams& p, cudaStream_t st) {
-  const size_t smem = sizeof(DBSmem<D>) + 1024;
-  static_assert(sizeof(DBSmem<D>) + 1024 <= 232448, "shared memory");
-  auto kern = fwd_db_kernel<D>;
+                const CUtensorMap& mb, const FwdParams& p, cudaStream_t st) {
+  const size_t smem = sizeof(DBSmem<D, BT>) + 1024;
+  static_assert(sizeof(DBSmem<D, BT>) + 1024 <= 232448, "shared memory");
+  auto kern = fwd_db_kernel<D, BT>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess)
     return ATTN_ERR_CUDA;
   const unsigned nblk = (g.Nq + 2 * BM - 1) / (2 * BM);
   const dim3 grid = p.batch_inner ? dim3(g.B, nblk, g.Hq) : dim3(nblk, g.Hq, g.B);
   if (grid.y > 65535 || grid.z > 65535) return ATTN_ERR_UNSUPPORTED;
   record_kernel_event(ATTN_KERNEL_FWD, 0, st);
-  kern<<<grid, kThreads, smem, st>>>(mq, mk, mv, p);
+  kern<<<grid, kThreadsOf<BT>, smem, st>>>(mq, mk, mv, mb, p);
   record_kernel_event(ATTN_KERNEL_FWD, 1, st);
   count_launch();
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;
@@ -455,8 +521,24 @@ int launch_fwd_db(const TcGeom& g, const CUtensorMap& mq, const CUtensorMap& mk,
                   const FwdParams& p, cudaStream_t st) {
   const int dv = g.Dv ? g.Dv : g.D;
   if (!g.bias || g.alibi || g.cu_q || p.num_splits != 1 || dv != g.D) return ATTN_ERR_UNSUPPORTED;
-  if (g.D == 128) return launch_db_t<128>(g, mq, mk, mv, p, st);
-  if (g.D == 64) return launch_db_t<64>(g, mq, mk, mv, p, st);
+  // bias rows staged by TMA when they can be: 16-byte aligned base, rows and
+  // batch stride (the same test as the vector loads); a 4-D view (key, query
+  // row, head, batch), one batch when the batch shares the bias
+  CUtensorMap mb;
+  std::memset(&mb, 0, sizeof(mb));
+  const bool bt = p.bias_vec4;
+  if (bt) {
+    const uint64_t hs = (uint64_t)g.Nq * g.Nk;
+    const uint64_t dims[4] = {(uint64_t)g.Nk, (uint64_t)g.Nq, (uint64_t)g.Hq, g.bias_bstride ? (uint64_t)g.B : 1};
+    const uint64_t str[3] = {(uint64_t)g.Nk * 4, hs * 4, (g.bias_bstride ? (uint64_t)g.bias_bstride : g.Hq * hs) * 4};
+    const uint32_t box[4] = {32, BM, 1, 1};
+    if (encode_tmap(&mb, g.bias, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dims, str, box) != ATTN_OK)
+      return ATTN_ERR_CUDA;
+  }
+  if (g.D == 128) return bt ? launch_db_t<128, true>(g, mq, mk, mv, mb, p, st)
+                            : launch_db_t<128, false>(g, mq, mk, mv, mb, p, st);
+  if (g.D == 64) return bt ? launch_db_t<64, true>(g, mq, mk, mv, mb, p, st)
+                           : launch_db_t<64, false>(g, mq, mk, mv, mb, p, st);
   return ATTN_ERR_UNSUPPORTED;
 }
 
