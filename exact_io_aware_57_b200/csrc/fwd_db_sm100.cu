@@ -10,8 +10,8 @@
 // and works on the current one ("Understanding FlashAttention Pt 1", contents
 // 5.5: overlap data movement, matrix products and the softmax).  Measured on
 // the grouped causal workload with its 2.1 GB fp32 bias this runs the forward
-// at 1.6x the 128-key two-tile kernel; without a bias tensor to read, the
-// 128-key kernel is faster and is used instead.
+// at about twice the speed of the 128-key two-tile kernel; without a bias
+// tensor to read, the 128-key kernel is faster and is used instead.
 //
 //   warps 0..3  softmax of query tile 0: thread r owns query row r (TMEM lane r)
 //   warps 4..7  softmax of query tile 1
