@@ -142,9 +142,10 @@ ATTN_DEVINL void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c,
 // MASK zeroes queries this key is hidden from (query i sees key kj iff
 // kj - lo_off <= i <= kj + hi_off, i.e. i + diag - win_l <= kj <= i + diag + win_r;
 // padding rows and keys).
+// bb: the dense bias of these 32 queries for this key (loaded ahead by the caller).
 template <bool MASK, int BIAS>
 ATTN_DEVINL void p_chunk(int c, const uint32_t (&sr)[32], uint32_t st_col, const float* nlse2, float scale_log2,
-                         const float* bcol, float neg_slope2, int nk, int i0, int len_q, int kj, int len_k,
+                         const float (&bb)[32], float neg_slope2, int i0, int len_q, int kj, int len_k,
                          int lo_off, int hi_off, int bias_diag, uint32_t (&pk)[16]) {
   const float4* nl4 = reinterpret_cast<const float4*>(nlse2 + c * 32);
   const int q0 = i0 + c * 32;
@@ -163,7 +164,7 @@ ATTN_DEVINL void p_chunk(int c, const uint32_t (&sr)[32], uint32_t st_col, const
     for (int u = 0; u < 4; ++u) {
       const int e = e4 * 4 + u;
       float t = fmaf(__uint_as_float(sr[e]), scale_log2, nlv[u]);
-      if constexpr (BIAS == kBiasDense) t = fmaf(__ldg(bcol + (long long)min(q0 + e, len_q - 1) * nk), kLog2e, t);
+      if constexpr (BIAS == kBiasDense) t = fmaf(bb[e], kLog2e, t);
       if constexpr (BIAS == kBiasAlibi) t = fmaf(neg_slope2, fabsf(static_cast<float>(kj - q0 - e - bias_diag)), t);
       // unmasked tiles (every t finite): one exponential in kBwdEmuEvery on the FMA pipe
       float pe = (!MASK && kBwdEmuEvery > 0 && e % kBwdEmuEvery == kBwdEmuEvery - 1) ? ex2_poly(t) : ex2(t);
@@ -185,8 +186,8 @@ ATTN_DEVINL void p_chunk(int c, const uint32_t (&sr)[32], uint32_t st_col, const
 // the same columns (p_chunk), so the two groups need not wait for each other.
 // keep: this thread's P^T as bf16 pairs (chunk 2g in [0,16), chunk 2g+1 in [16,32)).
 template <bool MASK, int BIAS>
-ATTN_DEVINL void bwd_p_half(int grp, uint32_t st_col, const float* nlse2, float scale_log2, const float* bcol,
-                            float neg_slope2, int nk, int i0, int len_q, int kj, int len_k, int lo_off, int hi_off,
+ATTN_DEVINL void bwd_p_half(int grp, uint32_t st_col, const float* nlse2, float scale_log2, const float (&bb)[64],
+                            float neg_slope2, int i0, int len_q, int kj, int len_k, int lo_off, int hi_off,
                             int bias_diag, uint32_t (&keep)[32]) {
   const int c0 = 2 * grp;
   uint32_t ra[32], rb[32];
@@ -195,10 +196,11 @@ ATTN_DEVINL void bwd_p_half(int grp, uint32_t st_col, const float* nlse2, float 
   tmem_wait_ld();
   reg_fence(ra);
   reg_fence(rb);
-  p_chunk<MASK, BIAS>(c0, ra, st_col, nlse2, scale_log2, bcol, neg_slope2, nk, i0, len_q, kj, len_k, lo_off, hi_off,
-                      bias_diag, *reinterpret_cast<uint32_t(*)[16]>(&keep[0]));
-  p_chunk<MASK, BIAS>(c0 + 1, rb, st_col, nlse2, scale_log2, bcol, neg_slope2, nk, i0, len_q, kj, len_k, lo_off,
-                      hi_off, bias_diag, *reinterpret_cast<uint32_t(*)[16]>(&keep[16]));
+  p_chunk<MASK, BIAS>(c0, ra, st_col, nlse2, scale_log2, *reinterpret_cast<const float(*)[32]>(&bb[0]), neg_slope2,
+                      i0, len_q, kj, len_k, lo_off, hi_off, bias_diag, *reinterpret_cast<uint32_t(*)[16]>(&keep[0]));
+  p_chunk<MASK, BIAS>(c0 + 1, rb, st_col, nlse2, scale_log2, *reinterpret_cast<const float(*)[32]>(&bb[32]),
+                      neg_slope2, i0, len_q, kj, len_k, lo_off, hi_off, bias_diag,
+                      *reinterpret_cast<uint32_t(*)[16]>(&keep[16]));
 }
 
 // Phase B -- dS^T = P^T (dP^T - D) from the bf16 P^T and dP^T, into the
@@ -565,6 +567,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int st = step % NSTQ;
       const int h = hk * G + step / per_head;
       const int i0 = (i_first + step % per_head) * BM;
+      // the dense bias of this key and the group's 64 queries, loaded before the
+      // wait for the scores so that its latency passes there (rows past the end
+      // read the last row; their P^T is masked)
+      float bb[64];
+      if constexpr (BIAS == kBiasDense) {
+        const float* bcol = p.bias + b * p.bias_bstride + (long long)h * p.Nq * p.Nk + min(kj, len_k - 1);
+        const int qg = i0 + 64 * grp;
+#pragma unroll
+        for (int e = 0; e < 64; ++e) bb[e] = __ldg(bcol + (long long)min(qg + e, len_q - 1) * p.Nk);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 64; ++e) bb[e] = 0.f;
+      }
       // S^T is in TMEM; q_full of this stage (LSE rows) completed before, and
       // do_full (D rows) before dP^T
       ok = __all_sync(0xffffffffu, mbar_wait(&s.st_full, step & 1, ab));
@@ -574,17 +589,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       // warp-collective tcgen05 instructions, so every lane must take the same one
       const bool need_mask = (n0 + BN > len_k) || (i0 + BM > len_q) || (n0 + BN - 1 > i0 + diag + p.win_r) ||
                              (n0 < i0 + BM - 1 + diag - p.win_l);
-      const float* bcol = nullptr;
-      if constexpr (BIAS == kBiasDense) bcol = p.bias + b * p.bias_bstride + (long long)h * p.Nq * p.Nk + min(kj, len_k - 1);
       float neg_slope2 = 0.f;
       if constexpr (BIAS == kBiasAlibi) neg_slope2 = -__ldg(p.alibi + h) * kLog2e;
       const uint32_t st_col = tmem + lane_off + kColST, dp_col = tmem + lane_off + kColDPT;
       if (need_mask)
-        bwd_p_half<true, BIAS>(grp, st_col, s.nlse2[st], p.scale_log2, bcol, neg_slope2, p.Nk, i0, len_q, kj, len_k,
+        bwd_p_half<true, BIAS>(grp, st_col, s.nlse2[st], p.scale_log2, bb, neg_slope2, i0, len_q, kj, len_k,
                                diag + p.win_r, p.win_l - diag, diag, keep);
       else
-        bwd_p_half<false, BIAS>(grp, st_col, s.nlse2[st], p.scale_log2, bcol, neg_slope2, p.Nk, i0, len_q, kj, len_k,
-                                0, 0, diag, keep);
+        bwd_p_half<false, BIAS>(grp, st_col, s.nlse2[st], p.scale_log2, bb, neg_slope2, i0, len_q, kj, len_k, 0, 0,
+                                diag, keep);
       tmem_wait_st();
       // P^T is in TMEM: the dV MMAs (and the next step's scores) may start
       tc_fence_before();
