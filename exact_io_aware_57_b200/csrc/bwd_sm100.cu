@@ -563,23 +563,26 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) mbar_arrive(&s.staged[st]);
       return true;
     };
-    for (int step = 0; step < n_steps; ++step) {
-      const int st = step % NSTQ;
-      const int h = hk * G + step / per_head;
-      const int i0 = (i_first + step % per_head) * BM;
-      // the dense bias of this key and the group's 64 queries, loaded before the
-      // wait for the scores so that its latency passes there (rows past the end
-      // read the last row; their P^T is masked)
-      float bb[64];
+    // the dense bias of this key and the group's 64 queries of step t, loaded a
+    // step ahead (before the previous step's dQ staging) so that its latency
+    // passes there (rows past the end read the last row; their P^T is masked)
+    float bb[64];
+    auto load_bias = [&](int t) {
       if constexpr (BIAS == kBiasDense) {
-        const float* bcol = p.bias + b * p.bias_bstride + (long long)h * p.Nq * p.Nk + min(kj, len_k - 1);
-        const int qg = i0 + 64 * grp;
+        const int ht = hk * G + t / per_head, qg = (i_first + t % per_head) * BM + 64 * grp;
+        const float* bcol = p.bias + b * p.bias_bstride + (long long)ht * p.Nq * p.Nk + min(kj, len_k - 1);
 #pragma unroll
         for (int e = 0; e < 64; ++e) bb[e] = __ldg(bcol + (long long)min(qg + e, len_q - 1) * p.Nk);
       } else {
 #pragma unroll
         for (int e = 0; e < 64; ++e) bb[e] = 0.f;
       }
+    };
+    if (n_steps > 0) load_bias(0);
+    for (int step = 0; step < n_steps; ++step) {
+      const int st = step % NSTQ;
+      const int h = hk * G + step / per_head;
+      const int i0 = (i_first + step % per_head) * BM;
       // S^T is in TMEM; q_full of this stage (LSE rows) completed before, and
       // do_full (D rows) before dP^T
       ok = __all_sync(0xffffffffu, mbar_wait(&s.st_full, step & 1, ab));
@@ -612,6 +615,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&s.ds_ready);
+      if (step + 1 < n_steps) load_bias(step + 1);
       if (!(ok = drain(step))) break;
     }
     // ---- epilogue: dV (columns [grp DV/2, grp DV/2 + DV/2)) and dK (scaled,
