@@ -107,13 +107,14 @@ ATTN_DEVINL bool packed_seq(const int* cu, int z, int total, int max_len, int* s
 // heavy units of all groups but the last start early and the last CTAs to start
 // are light (a short tail), while the CTAs running at one time span few heads
 // and share their K/V (or Q/dO) tiles in L2.
-ATTN_DEVINL void grouped_unit(int nr, int nu, int gs, int& r, int& u) {
-  const int i = (int)(blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z));
+ATTN_DEVINL void grouped_unit_at(int i, int nr, int nu, int gs, int& r, int& u) {
   const int g = i / (gs * nr), base = g * gs, gn = min(gs, nu - base);
   const int rem = i - g * gs * nr;
   r = rem / gn;
   u = base + rem % gn;
 }
+ATTN_DEVINL int linear_block() { return (int)(blockIdx.x + gridDim.x * (blockIdx.y + gridDim.y * blockIdx.z)); }
+ATTN_DEVINL void grouped_unit(int nr, int nu, int gs, int& r, int& u) { grouped_unit_at(linear_block(), nr, nu, gs, r, u); }
 
 // ------------------------------------------------------------------------- TMA
 ATTN_DEVINL void tma_prefetch_desc(const CUtensorMap* map) {

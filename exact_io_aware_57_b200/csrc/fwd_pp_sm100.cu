@@ -42,6 +42,8 @@
 // each CTA then writes O_t (normalised, fp32) and LSE_t for the merge.
 #include <algorithm>
 
+#include <climits>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -144,8 +146,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   // every batch element of two heads, so the ones reading the same bias rows
   // run side by side
   const bool bi = !PARTIAL && p.batch_inner;
-  const int nblk = bi ? (int)gridDim.y : (int)gridDim.x;
-  int blk_raw, h, z;
+  const int nblk = bi ? (int)gridDim.y : PARTIAL ? (int)gridDim.x : p.grid_nblk;
+  int blk_raw, h, z, half = -1;  // half >= 0: this CTA takes only that 128-row tile of its unit
   if (PARTIAL) {
     blk_raw = blockIdx.x, h = blockIdx.y, z = blockIdx.z / p.num_splits;
   } else if (bi) {
@@ -154,8 +156,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     grouped_unit(nblk, nb * p.Hq, 2 * nb, blk_raw, u);
     h = u / nb, z = u % nb;
   } else {
-    int u;
-    grouped_unit(nblk, (int)(gridDim.y * gridDim.z), 8, blk_raw, u);
+    int unit = linear_block(), u;
+    if (unit >= p.half_from) {
+      half = (unit - p.half_from) & 1;
+      unit = p.half_from + ((unit - p.half_from) >> 1);
+    }
+    grouped_unit_at(unit, nblk, p.grid_nu, 8, blk_raw, u);
     h = u % p.Hq, z = u / p.Hq;
   }
   const int blk = p.causal ? nblk - 1 - blk_raw : blk_raw;
@@ -168,7 +174,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       return;
     bidx = 0;
   }
-  const int m0 = blk * 2 * BM;
+  const int m0 = blk * 2 * BM + (half > 0 ? BM : 0);
   if (m0 >= len_q) return;  // uniform: before any barrier or TMEM use
   const int hk = h / (p.Hq / p.Hkv);
   const int diag = len_k - len_q;  // row i is aligned with key i + diag
@@ -177,6 +183,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   TileRange rg[2];
   rg[0] = tile_range(m0, len_q, diag, p.win_l, p.win_r, k_lo, k_hi);
   rg[1] = tile_range(m0 + BM, len_q, diag, p.win_l, p.win_r, k_lo, k_hi);
+  if (half >= 0) rg[1] = TileRange{0, 0};  // a single tile
   // union of the two ranges (contiguous: each tile's band overlaps the next)
   const int J0 = rg[0].n > 0 ? rg[0].jb : rg[1].jb;
   const int J1 = rg[1].n > 0 ? rg[1].jb + rg[1].n : rg[0].jb + rg[0].n;
@@ -316,7 +323,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int r = quarter * 32 + lane;
     const int mt = m0 + t * BM;
     const int i = mt + r;  // row inside its sequence
-    const bool row_ok = i < len_q;
+    // a CTA that takes a single tile (half >= 0) owns no rows of tile 1: those
+    // belong to the CTA of the other half (or the next row block)
+    const bool row_ok = i < len_q && !(half >= 0 && t == 1);
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t col_s = tmem + lane_off + t * 128, col_o = tmem + lane_off + 256 + t * DV;
     const TileRange my = t ? rg[1] : rg[0];
@@ -533,10 +542,25 @@ int launch_pp_t(const TcGeom& g, const CUtensorMap& mq, const CUtensorMap& mk, c
     return ATTN_ERR_CUDA;
   const int max_nq = g.cu_q ? g.max_nq : g.Nq;
   const unsigned nblk = (max_nq + 2 * BM - 1) / (2 * BM), nz = (g.cu_q ? g.num_seqs : g.B) * p.num_splits;
-  const dim3 grid = (!PARTIAL && p.batch_inner) ? dim3(nz, nblk, g.Hq) : dim3(nblk, g.Hq, nz);
+  dim3 grid = (!PARTIAL && p.batch_inner) ? dim3(nz, nblk, g.Hq) : dim3(nblk, g.Hq, nz);
   if (grid.y > 65535 || grid.z > 65535) return ATTN_ERR_UNSUPPORTED;
+  FwdParams q = p;
+  const long long units = (long long)nblk * g.Hq * nz;
+  q.grid_nblk = (int)nblk;
+  q.grid_nu = g.Hq * (int)nz;
+  q.half_from = (int)std::min<long long>(units, INT_MAX);
+  // Equal units (no causal mask, no window, dense batches) in one CTA per SM:
+  // when the last wave would fill at most half the SMs, its units run as single
+  // 128-row tiles, two CTAs each, and the wave ends sooner.
+  if (!PARTIAL && !p.batch_inner && !g.cu_q && !g.causal && g.window_left < 0 && g.window_right < 0) {
+    const long long sms = sm_count(), tail = units % sms;
+    if (units >= sms && tail > 0 && 2 * tail <= sms && units + tail < INT_MAX) {
+      q.half_from = (int)(units - tail);
+      grid = dim3((unsigned)(units + tail));
+    }
+  }
   record_kernel_event(ATTN_KERNEL_FWD, 0, st);
-  kern<<<grid, kThreads, smem, st>>>(mq, mk, mv, p);
+  kern<<<grid, kThreads, smem, st>>>(mq, mk, mv, q);
   record_kernel_event(ATTN_KERNEL_FWD, 1, st);
   count_launch();
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ERR_CUDA;

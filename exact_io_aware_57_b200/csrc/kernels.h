@@ -21,6 +21,8 @@ constexpr long long kWaitLimitCycles = 2000000000LL;
 
 // Device address of the library's status word on the current device.
 int* device_status_ptr();
+// Streaming multiprocessors of the current device (1 if the query fails).
+int sm_count();
 
 // ----------------------------------------------------------------- fp32 path
 // Key visibility.  With a = i + Nk - Nq the key aligned with query row i, key j
@@ -106,6 +108,11 @@ struct FwdParams {
   const float* k_scale;
   int* status;
   long long wait_limit;
+  // Two-tile forward, dense grid (set by its launcher): grid_nblk row blocks of
+  // 256 rows x grid_nu (batch, head) pairs.  Units from half_from on (in launch
+  // order) are split into their two 128-row tiles, one CTA each, so that a last
+  // wave that would leave SMs idle runs single tiles instead (a 1-D grid).
+  int grid_nblk, grid_nu, half_from;
 };
 
 // Forward with two 128-row query tiles per CTA whose softmax warpgroups

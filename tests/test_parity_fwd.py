@@ -39,6 +39,13 @@ def test_fwd_bf16_ragged_head_groups(orc):
     check_fwd(orc, 3, 4, 2, 600, 600, 128, True, seed=11)
 
 
+def test_fwd_bf16_tail_wave_single_tiles(orc):
+    """52 heads x 3 row blocks = 156 equal units on 148 SMs: the last 8 run as
+    single 128-row tiles, two CTAs each, among them the ragged last row block
+    (one of its CTAs has no rows at all)."""
+    check_fwd(orc, 1, 52, 4, 600, 600, 64, False, seed=13)
+
+
 def test_fwd_bf16_peaked_scores(orc):
     """Q, K ~ N(0, 3^2): frequent running-max rescales (the causal fwd+bwd workload's regime)."""
     check_fwd(orc, 1, 2, 2, 1024, 1024, 128, True, sigma=3.0)
