@@ -40,8 +40,9 @@
 // nested at their ends, and each tile walks only its own.
 // Split-KV: with num_splits > 1 the grid's z index also runs over key ranges;
 // each CTA then writes O_t (normalised, fp32) and LSE_t for the merge.
+// With equal units, a last wave that would fill at most half the SMs runs its
+// 256-row units as single 128-row tiles, one CTA each (FwdParams::half_from).
 #include <algorithm>
-
 #include <climits>
 
 #include "common.cuh"
