@@ -56,6 +56,13 @@ def test_bwd_bf16_bias_gqa(orc):
     check_bwd(orc, 2, 4, 2, 257, 257, 128, True, bias=True)
 
 
+@pytest.mark.parametrize("Nq,Nk", [(300, 500), (500, 300)])
+def test_bwd_bf16_bias_unequal_lengths(orc, Nq, Nk):
+    """Dense bias with bottom-right aligned causal lengths (bias values loaded a
+    step ahead, clamped at the last row)."""
+    check_bwd(orc, 1, 4, 2, Nq, Nk, 128, True, bias=True, seed=15)
+
+
 def test_bwd_bf16_bias_shared_three_batches(orc):
     """A bias shared by three batch elements: their CTAs run side by side
     (batch-innermost grid); rows of 388 keys with a ragged last tile."""

@@ -57,6 +57,13 @@ def test_fwd_bf16_bias_gqa(orc, per_batch):
     check_fwd(orc, 2, 4, 2, 257, 257, 128, True, bias=True, per_batch_bias=per_batch)
 
 
+@pytest.mark.parametrize("Nq,Nk", [(300, 500), (500, 300)])
+def test_fwd_bf16_bias_unequal_lengths(orc, Nq, Nk):
+    """Dense bias (rows of Nk = 0 mod 4 floats: staged by TMA) with bottom-right
+    aligned causal lengths: a ragged last key tile and, for Nq > Nk, rows with no key."""
+    check_fwd(orc, 2, 4, 2, Nq, Nk, 128, True, bias=True, seed=14)
+
+
 def test_fwd_bf16_bias_noncausal_d64(orc):
     check_fwd(orc, 1, 2, 1, 190, 190, 64, False, bias=True)
 
