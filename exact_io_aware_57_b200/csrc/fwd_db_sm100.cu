@@ -524,16 +524,16 @@ int launch_fwd_db(const TcGeom& g, const CUtensorMap& mq, const CUtensorMap& mk,
   // bias rows staged by TMA when they can be: 16-byte aligned base, rows and
   // batch stride (the same test as the vector loads); a 4-D view (key, query
   // row, head, batch), one batch when the batch shares the bias
+  // (a view the tensor map cannot describe falls back to the direct loads)
   CUtensorMap mb;
   std::memset(&mb, 0, sizeof(mb));
-  const bool bt = p.bias_vec4;
+  bool bt = p.bias_vec4;
   if (bt) {
     const uint64_t hs = (uint64_t)g.Nq * g.Nk;
     const uint64_t dims[4] = {(uint64_t)g.Nk, (uint64_t)g.Nq, (uint64_t)g.Hq, g.bias_bstride ? (uint64_t)g.B : 1};
     const uint64_t str[3] = {(uint64_t)g.Nk * 4, hs * 4, (g.bias_bstride ? (uint64_t)g.bias_bstride : g.Hq * hs) * 4};
     const uint32_t box[4] = {32, BM, 1, 1};
-    if (encode_tmap(&mb, g.bias, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dims, str, box) != ATTN_OK)
-      return ATTN_ERR_CUDA;
+    bt = encode_tmap(&mb, g.bias, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, dims, str, box) == ATTN_OK;
   }
   if (g.D == 128) return bt ? launch_db_t<128, true>(g, mq, mk, mv, mb, p, st)
                             : launch_db_t<128, false>(g, mq, mk, mv, mb, p, st);
